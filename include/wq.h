@@ -1,0 +1,145 @@
+/*
+ * wq.h - C ABI of libwq: round-to-nearest group-wise affine INT4 weight quantization
+ * and the W4A16 dequant-matmul, for NVIDIA B200 (sm_100a).
+ *
+ * Definitions followed (page title, section):
+ *   "Model Quantization", 1 "Mathematical Mechanics of Quantization": affine
+ *      W_q = round(W/S) + Z, W_dequant = S (W_q - Z); one S and Z per group of g = 128.
+ *   "DL S067 - Quantization", 1 "The core math": asymmetric
+ *      S = (beta - alpha)/(q_max - q_min), Z = round(q_min - alpha/S),
+ *      q = clip(round(W/S) + Z, q_min, q_max); symmetric S = max|W|/q_max.
+ *   "DL S067 - Quantization", 2 "Per-tensor vs per-channel vs per-group": a group is g
+ *      consecutive weights along the input dimension of W [out_features, in_features].
+ *   "LLM Weight Quantization - GPTQ, AWQ, SmoothQuant, FP8 & INT4/INT8 Trade-offs",
+ *      "The vocabulary": W4A16 = 4-bit weights dequantized to 16 bits inside the kernel,
+ *      16-bit matmul (here: bf16 operands, fp32 accumulation), Y = X W^T.
+ *
+ * Numerics fixed by this library (the pages leave them open):
+ *   - alpha = min(0, min w), beta = max(0, max w) over the group (zero is exact);
+ *   - S' = binary16 round-half-even of the EXACT (beta - alpha)/15; S' = 0 -> 1.0;
+ *   - Z = clip(round-half-even(-alpha/S'), 0, 15) on the exact quotient, stored binary16;
+ *   - q = clip(round-half-even(w/S') + Z, 0, 15) on the exact quotient;
+ *   - INT8 symmetric: s' = binary16(max|w|/127), q = clip(RNE(w/s'), -127, 127).
+ *
+ * Data layout (row-major, all device memory owned by the caller):
+ *   W      [N, K] fp32 or bf16, leading dimension ldw elements (N = out, K = in)
+ *   packed [N, K/2] uint8: byte j of row n = q[n][2j] | q[n][2j+1] << 4
+ *   S, Z   [N, K/g] binary16 bit patterns (uint16), contiguous
+ *   X      [M, K] bf16, leading dimension ldx; Y [M, N] bf16, leading dimension ldy
+ *
+ * Conventions:
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless stated.
+ *     The library allocates no device memory; a small device status word and the
+ *     kernels' code are module globals.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *     legacy default stream) on the current device.
+ *   - Argument errors are returned synchronously and launch nothing. A failed launch
+ *     returns WQ_ERR_CUDA. Data-dependent errors (non-finite weights, scale overflow,
+ *     codes > 15, a bounded wait that timed out) are recorded in the device status word
+ *     and returned by wq_get_status(); outputs of such a call are unspecified.
+ *   - Thread-safe for distinct streams; calls on one stream are ordered.
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WQ_VERSION 100 /* 0.1.0 */
+
+typedef enum wq_status {
+  WQ_OK = 0,
+  WQ_ERR_NULL = 1,        /* a required pointer is NULL                          */
+  WQ_ERR_SHAPE = 2,       /* sizes <= 0, K % g != 0, K odd, ld too small, ...    */
+  WQ_ERR_ALIGN = 3,       /* a pointer or leading dimension breaks 16-B alignment */
+  WQ_ERR_DTYPE = 4,       /* dtype not supported by this call                    */
+  WQ_ERR_UNSUPPORTED = 5, /* parameter combination not implemented               */
+  WQ_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed                */
+  WQ_ERR_NONFINITE = 7,   /* device: NaN/inf weight or binary16 scale overflow   */
+  WQ_ERR_TIMEOUT = 8,     /* device: a bounded barrier wait gave up              */
+  WQ_ERR_RANGE = 9,       /* device: a code given to wq_pack_int4 exceeds 15     */
+  WQ_ERR_NODEVICE = 10    /* no CUDA device, or it is not sm_100                 */
+} wq_status;
+
+typedef enum wq_dtype { WQ_F32 = 0, WQ_BF16 = 1, WQ_F16 = 2, WQ_U8 = 3, WQ_I8 = 4 } wq_dtype;
+
+/* Quantization parameters, named after the usual config keys (w_bit, q_group_size,
+ * zero_point). Supported: {4, g, 1} with g a multiple of 32 that divides K (g = K is
+ * per output channel), and {8, K, 0} (INT8 symmetric per channel). */
+typedef struct wq_qparams {
+  int32_t w_bit;      /* 4 or 8                                      */
+  int32_t group;      /* g: weights per scale along K                 */
+  int32_t zero_point; /* 1 = asymmetric [0, 15]; 0 = symmetric        */
+} wq_qparams;
+
+/* Library version (WQ_VERSION) and a static description of a status code. */
+int32_t wq_version(void);
+const char* wq_status_string(wq_status status);
+
+/* Round-to-nearest quantization of W [N, K] ("DL S067 - Quantization", sections 1-2).
+ *   W       fp32 or bf16 (w_dtype), row stride ldw >= K elements; base and row stride
+ *           16-byte aligned.
+ *   params  NULL means {4, 128, 1}.
+ *   INT4 ({4, g, 1}): packed [N, K/2] uint8, S and Z [N, K/g] binary16.
+ *   INT8 ({8, K, 0}): packed receives int8 codes [N, K]; S [N] binary16; Z must be NULL.
+ * Non-finite weights or a scale above the binary16 range set WQ_ERR_NONFINITE in the
+ * device status word. Requires K % 32 == 0. */
+wq_status wq_quantize_rtn_g128(const void* W, wq_dtype w_dtype, int64_t N, int64_t K,
+                               int64_t ldw, const wq_qparams* params, uint8_t* packed,
+                               uint16_t* S, uint16_t* Z, void* stream);
+
+/* Per-tensor asymmetric INT4 (one S, Z for all of W; same page, section 2). Two passes:
+ * a min/max reduction into the caller's `workspace` (device memory of at least
+ * wq_quantize_per_tensor_workspace_bytes(N, K) bytes, 16-byte aligned, no initial
+ * contents required), then the codes. S and Z each receive one binary16 value. */
+size_t wq_quantize_per_tensor_workspace_bytes(int64_t N, int64_t K);
+wq_status wq_quantize_rtn_per_tensor(const void* W, wq_dtype w_dtype, int64_t N,
+                                     int64_t K, int64_t ldw, uint8_t* packed, uint16_t* S,
+                                     uint16_t* Z, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/* Pack 4-bit codes two per byte (the storage of "INT4 weights + FP16 scales/zero-points",
+ * "Model Quantization", section 4): codes [N, K] uint8 in [0, 15] -> packed [N, K/2].
+ * A code above 15 sets WQ_ERR_RANGE in the status word. Requires K % 32 == 0. */
+wq_status wq_pack_int4(const uint8_t* codes, int64_t N, int64_t K, uint8_t* packed,
+                       void* stream);
+
+/* Dequantize W_hat = S' (q - Z) ("Model Quantization", section 1) into out [N, K]:
+ * WQ_F32 is exact; WQ_BF16 is its round-half-even to bfloat16. group = g as above, or
+ * 0 for per-tensor (S, Z hold one value). Requires K % 32 == 0. */
+wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z,
+                     int64_t N, int64_t K, int32_t group, void* out, wq_dtype out_dtype,
+                     void* stream);
+
+/* W4A16 matmul Y = X W_hat^T ("LLM Weight Quantization ...", "The vocabulary"):
+ *   X [M, K] bf16 (ldx), packed/S/Z as produced above with group g (0 = per-tensor),
+ *   Y [M, N] bf16 (ldy), fp32 accumulation.
+ * Kernel choice by M: M <= 8 streams the packed weights on CUDA cores with the
+ * dequantization in registers and S' factored out of each group (exact S'(q - Z));
+ * larger M runs the tensor-core GEMM, which dequantizes each weight tile to bf16 in
+ * shared memory (so W_hat is rounded to bfloat16 there).
+ * Requires K % 128 == 0 for M > 8; K % 32 == 0 otherwise; ldx, ldy multiples of 8. */
+wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* packed,
+                        const uint16_t* S, const uint16_t* Z, int64_t N, int64_t K,
+                        int32_t group, uint16_t* Y, int64_t ldy, void* stream);
+
+/* W8A16 matmul with INT8 symmetric per-channel weights: codes int8 [N, K], S [N]
+ * binary16; Y = X (s' q)^T, fp32 accumulation, bf16 out. Same M rules as above. */
+wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t* codes,
+                        const uint16_t* S, int64_t N, int64_t K, uint16_t* Y, int64_t ldy,
+                        void* stream);
+
+/* Synchronize `stream`, then return and clear the current device's status word:
+ * WQ_OK, or the first of WQ_ERR_NONFINITE / WQ_ERR_RANGE / WQ_ERR_TIMEOUT recorded by a
+ * kernel since the last call; WQ_ERR_CUDA if the synchronization itself failed. */
+wq_status wq_get_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H_ */

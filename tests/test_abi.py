@@ -1,0 +1,113 @@
+"""The C-ABI library builds, loads and exports every function include/wq.h declares, and its
+host-side argument checks reject bad calls before touching a device (CPU only: no kernel
+runs, and the fake pointers passed here are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a16_dequant_matmul_b200 as wq
+from w4a16_dequant_matmul_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wq.h")
+
+OK, NULL, SHAPE, ALIGN, DTYPE, UNSUP, NODEV = 0, 1, 2, 3, 4, 5, 10
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+ODD = ctypes.c_void_p(0x10008)       # 8-byte but not 16-byte aligned
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build_library()
+    return wq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("wq_quantize_rtn_g128", "wq_pack_int4", "wq_dequant", "wq_w4a16_gemm"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(wq._SIGNATURES), "binding must wrap every C entry point"
+
+
+def test_version_and_status_strings(lib):
+    assert wq.wq_version() == 100
+    for code in range(11):
+        s = wq.wq_status_string(code)
+        assert s and s != "unknown status"
+    assert wq.wq_status_string(99) == "unknown status"
+
+
+def _qp(w_bit=4, group=128, zp=1):
+    return ctypes.byref(wq._QParams(w_bit, group, zp))
+
+
+def test_quantize_argument_checks(lib):
+    f = lib.wq_quantize_rtn_g128
+    # empty problems are a no-op
+    assert f(None, wq.WQ_BF16, 0, 128, 128, None, None, None, None, None) == OK
+    assert f(FAKE, wq.WQ_BF16, -1, 128, 128, None, FAKE, FAKE, FAKE, None) == SHAPE
+    assert f(FAKE, wq.WQ_F16, 4, 128, 128, None, FAKE, FAKE, FAKE, None) == DTYPE
+    assert f(None, wq.WQ_BF16, 4, 128, 128, None, FAKE, FAKE, FAKE, None) == NULL
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 128, None, FAKE, FAKE, None, None) == NULL
+    assert f(FAKE, wq.WQ_BF16, 4, 100, 128, None, FAKE, FAKE, FAKE, None) == SHAPE   # K % 32
+    assert f(FAKE, wq.WQ_BF16, 4, 192, 192, None, FAKE, FAKE, FAKE, None) == SHAPE   # K % g
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 64, None, FAKE, FAKE, FAKE, None) == SHAPE    # ldw < K
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(4, 48), FAKE, FAKE, FAKE, None) == SHAPE
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(3, 128), FAKE, FAKE, FAKE, None) == UNSUP
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(8, 128, 0), FAKE, FAKE, FAKE, None) == UNSUP
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(8, 64, 0), FAKE, FAKE, None, None) == UNSUP
+    assert f(ODD, wq.WQ_BF16, 4, 128, 128, None, FAKE, FAKE, FAKE, None) == ALIGN
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 132, None, FAKE, FAKE, FAKE, None) == ALIGN   # row stride
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 128, None, ODD, FAKE, FAKE, None) == ALIGN
+
+
+def test_gemm_argument_checks(lib):
+    g = lib.wq_w4a16_gemm
+    assert g(FAKE, 0, 128, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 64, None) == OK    # M = 0
+    assert g(FAKE, 1, 128, FAKE, FAKE, FAKE, 0, 128, 128, FAKE, 64, None) == OK     # N = 0
+    assert g(FAKE, 1, 128, FAKE, FAKE, FAKE, 64, 0, 128, FAKE, 64, None) == SHAPE   # K = 0
+    assert g(None, 1, 128, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 64, None) == NULL
+    assert g(FAKE, 1, 128, FAKE, FAKE, None, 64, 128, 128, FAKE, 64, None) == NULL
+    assert g(FAKE, 1, 96, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 64, None) == SHAPE  # ldx < K
+    assert g(FAKE, 2, 128, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 32, None) == SHAPE # ldy < N
+    assert g(FAKE, 1, 128, FAKE, FAKE, FAKE, 64, 128, 96, FAKE, 64, None) == SHAPE  # K % g
+    assert g(FAKE, 1, 132, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 64, None) == ALIGN # ldx % 8
+    assert g(ODD, 1, 128, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 64, None) == ALIGN
+    h = lib.wq_w8a16_gemm
+    assert h(FAKE, 1, 128, None, FAKE, 64, 128, FAKE, 64, None) == NULL
+    assert h(FAKE, 1, 128, FAKE, FAKE, 64, 100, FAKE, 64, None) == SHAPE
+
+
+def test_pack_dequant_argument_checks(lib):
+    assert lib.wq_pack_int4(FAKE, 4, 100, FAKE, None) == SHAPE
+    assert lib.wq_pack_int4(None, 4, 128, FAKE, None) == NULL
+    assert lib.wq_pack_int4(ODD, 4, 128, FAKE, None) == ALIGN
+    d = lib.wq_dequant
+    assert d(FAKE, FAKE, FAKE, 4, 128, 128, FAKE, wq.WQ_F16, None) == DTYPE
+    assert d(FAKE, FAKE, FAKE, 4, 128, 48, FAKE, wq.WQ_F32, None) == SHAPE
+    assert d(FAKE, None, FAKE, 4, 128, 128, FAKE, wq.WQ_F32, None) == NULL
+    p = lib.wq_quantize_rtn_per_tensor
+    assert p(FAKE, wq.WQ_BF16, 4, 128, 128, FAKE, FAKE, FAKE, None, 0, None) == NULL
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="host without a GPU only")
+def test_valid_call_without_device_reports_nodevice(lib):
+    """A call that passes every host check but finds no sm_100 device fails loudly
+    (WQ_ERR_NODEVICE), and the Python binding raises: there is no CPU fallback."""
+    assert lib.wq_w4a16_gemm(FAKE, 1, 128, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 64, None) == NODEV
+    assert lib.wq_get_status(None) in (NODEV, 6)

@@ -1,0 +1,118 @@
+"""GPU parity of the W4A16 / W8A16 matmul against the float64 oracle on the same
+dequantized weights. Gate: max |y - y_ref| / max(|y_ref|, 1e-3 rms(y_ref)) <= 1e-2
+(bf16 output rounding is 2^-9 relative; fp32 accumulation adds ~1e-6)."""
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import oracle  # noqa: E402
+import w4a16_dequant_matmul_b200 as wq  # noqa: E402
+import wq_inputs  # noqa: E402
+from tests import gpu_util as gu  # noqa: E402
+
+GATE = 1e-2
+
+
+def _quantize_both(Wb, group):
+    """GPU quantization of bf16 W and the oracle's; asserts they agree bit for bit."""
+    Wt = gu.bf16_from_bits(Wb)
+    if group == 0:
+        packed, S, Z = wq.wq_quantize_rtn_per_tensor(Wt)
+    else:
+        packed, S, Z = wq.wq_quantize_rtn_g128(Wt, 4, group, True)
+    codes, So, Zo = oracle.quantize_rtn_asym(wq_inputs.bf16_bits_to_f64(Wb), group)
+    np.testing.assert_array_equal(gu.to_np(packed), oracle.pack_int4(codes))
+    np.testing.assert_array_equal(gu.bits16(S).ravel(), gu.f16_bits_of(So).ravel())
+    return packed, S, Z, codes, So, Zo
+
+
+def test_tiny_config():
+    """W fp32 256x512, X bf16 1x512: Y 1x256 against the oracle."""
+    W, Xb = wq_inputs.tiny_config()
+    packed, S, Z = wq.wq_quantize_rtn_g128(gu.f32(W))
+    codes, So, Zo = oracle.quantize_rtn_asym(W.astype(np.float64), 128)
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "exact")
+    assert Y.shape == (1, 256)
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE
+
+
+SHAPES = [(256, 512), (300, 1152), (1000, 4096), (77, 2304), (129, 11008)]
+
+
+@pytest.mark.parametrize("N,K", SHAPES)
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 8])
+def test_small_m_parity(N, K, M):
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + K)
+    Xb = wq_inputs.act_bf16(M, K, seed=M)
+    packed, S, Z, codes, So, Zo = _quantize_both(Wb, 128)
+    X = gu.bf16_from_bits(Xb)
+    Y = wq.wq_w4a16_gemm(X, packed, S, Z, 128)
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "exact")
+    y = gu.bf16_to_f64(Y)
+    assert oracle.gemm_gate(y, Yref) <= GATE
+    assert oracle.rel_frobenius(Yref, y) < 4e-3
+    Y2 = wq.wq_w4a16_gemm(X, packed, S, Z, 128)
+    assert torch.equal(Y, Y2), "fixed reduction order: repeated runs are bitwise identical"
+
+
+@pytest.mark.parametrize("group", [32, 256, 2304, 0])
+@pytest.mark.parametrize("M", [1, 4])
+def test_granularities(group, M):
+    Wb, Xb, _ = wq_inputs.outlier_config(N=96, K=2304, M=M)
+    packed, S, Z, codes, So, Zo = _quantize_both(Wb, group)
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, group)
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, group, "exact")
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE
+
+
+def test_strided_x_and_y():
+    N, K, M = 200, 1024, 3
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=9)
+    Xwide = gu.bf16_from_bits(wq_inputs.act_bf16(M, K + 64, seed=2))
+    X = Xwide[:, 64:]
+    packed, S, Z, codes, So, Zo = _quantize_both(Wb, 128)
+    Ybig = torch.full((M, N + 40), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Y = Ybig[:, 8:8 + N]
+    wq.wq_w4a16_gemm(X, packed, S, Z, 128, Y=Y)
+    Yref = oracle.w4a16_matmul(gu.bf16_to_f64(X), codes, So, Zo, 128, "exact")
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE
+    assert torch.isnan(Ybig[:, :8]).all() and torch.isnan(Ybig[:, 8 + N:]).all()
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (11008, 4096), (4096, 11008)])
+def test_full_size_decode_sampled(N, K):
+    """7B-class layer shapes at M = 1 in the benchmark's configuration: GPU quantization
+    of the whole W, GEMV over all N rows; the oracle quantizes and multiplies 64 sampled
+    rows on its own."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.02)
+    Xb = wq_inputs.act_bf16(1, K)
+    Wt = gu.bf16_from_bits(Wb)
+    packed, S, Z = wq.wq_quantize_rtn_g128(Wt)
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    rows = np.sort(np.random.default_rng(N + K).choice(N, 64, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    codes, So, Zo = oracle.quantize_rtn_asym(wq_inputs.bf16_bits_to_f64(Wb[rows]), 128)
+    np.testing.assert_array_equal(gu.to_np(packed)[rows], oracle.pack_int4(codes))
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "exact")
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref) <= GATE
+
+
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_w8a16_small_m(M):
+    N, K = 130, 2048
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=11)
+    Xb = wq_inputs.act_bf16(M, K, seed=12)
+    q, S, _ = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb), 8, K, False)
+    qo, so = oracle.quantize_sym_int8_per_channel(wq_inputs.bf16_bits_to_f64(Wb))
+    np.testing.assert_array_equal(gu.to_np(q), qo)
+    Y = wq.wq_w8a16_gemm(gu.bf16_from_bits(Xb), q, S)
+    Yref = oracle.w8a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), qo, so, "exact")
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE

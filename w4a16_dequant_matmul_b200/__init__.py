@@ -1,0 +1,246 @@
+"""Python binding of libwq, the B200 (sm_100a) library for round-to-nearest group-wise INT4
+weight quantization and the W4A16 dequant-matmul.
+
+Argument marshalling only: every function forwards device pointers of torch tensors to the
+C ABI declared in include/wq.h, on the current CUDA stream; all arithmetic runs in the
+library's kernels. There is no CPU path: without libwq.so or a CUDA device the calls raise.
+
+Functions carry the C names:
+    wq_quantize_rtn_g128(W, w_bit=4, group=128, zero_point=True) -> (packed, S, Z)
+    wq_quantize_rtn_per_tensor(W) -> (packed, S, Z)
+    wq_pack_int4(codes) -> packed
+    wq_dequant(packed, S, Z, group, out_dtype) -> W_hat
+    wq_w4a16_gemm(X, packed, S, Z, group) -> Y
+    wq_w8a16_gemm(X, codes, S) -> Y
+    wq_get_status() -> int
+S and Z are returned as torch.float16 tensors (binary16 bit patterns in the C ABI).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from ._build import LIB_PATH, build_library  # noqa: F401  (build_library re-exported)
+
+__all__ = [
+    "WQError", "lib", "status_name",
+    "wq_version", "wq_status_string", "wq_quantize_rtn_g128", "wq_quantize_rtn_per_tensor",
+    "wq_quantize_per_tensor_workspace_bytes", "wq_pack_int4", "wq_dequant", "wq_w4a16_gemm",
+    "wq_w8a16_gemm", "wq_get_status",
+    "WQ_F32", "WQ_BF16", "WQ_F16", "WQ_U8", "WQ_I8",
+]
+
+WQ_F32, WQ_BF16, WQ_F16, WQ_U8, WQ_I8 = 0, 1, 2, 3, 4
+STATUS_NAMES = {
+    0: "WQ_OK", 1: "WQ_ERR_NULL", 2: "WQ_ERR_SHAPE", 3: "WQ_ERR_ALIGN", 4: "WQ_ERR_DTYPE",
+    5: "WQ_ERR_UNSUPPORTED", 6: "WQ_ERR_CUDA", 7: "WQ_ERR_NONFINITE", 8: "WQ_ERR_TIMEOUT",
+    9: "WQ_ERR_RANGE", 10: "WQ_ERR_NODEVICE",
+}
+
+
+class WQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_name(status)} ({_raw_status_string(status)})")
+
+
+class _QParams(ctypes.Structure):
+    _fields_ = [("w_bit", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("zero_point", ctypes.c_int32)]
+
+
+_LIB = None
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+
+_SIGNATURES = {
+    "wq_version": (_I32, []),
+    "wq_status_string": (ctypes.c_char_p, [_I32]),
+    "wq_quantize_rtn_g128": (_I32, [_P, _I32, _I64, _I64, _I64, ctypes.POINTER(_QParams), _P, _P,
+                                    _P, _P]),
+    "wq_quantize_per_tensor_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "wq_quantize_rtn_per_tensor": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P,
+                                          ctypes.c_size_t, _P]),
+    "wq_pack_int4": (_I32, [_P, _I64, _I64, _P, _P]),
+    "wq_dequant": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _I32, _P]),
+    "wq_w4a16_gemm": (_I32, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I32, _P, _I64, _P]),
+    "wq_w8a16_gemm": (_I32, [_P, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _P]),
+    "wq_get_status": (_I32, [_P]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libwq.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m w4a16_dequant_matmul_b200._build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = handle
+    return _LIB
+
+
+def status_name(status: int) -> str:
+    return STATUS_NAMES.get(int(status), f"status {status}")
+
+
+def _raw_status_string(status: int) -> str:
+    try:
+        return lib().wq_status_string(int(status)).decode()
+    except Exception:  # the library itself may be what failed to load
+        return "?"
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise WQError(status, where)
+
+
+def _stream(stream=None):
+    import torch
+
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _rows(t, name):
+    if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
+    return t.stride(0) if t.shape[0] > 1 else max(t.shape[1], t.stride(0))
+
+
+def _w_dtype(t):
+    import torch
+
+    if t.dtype == torch.float32:
+        return WQ_F32
+    if t.dtype == torch.bfloat16:
+        return WQ_BF16
+    raise TypeError("W must be float32 or bfloat16")
+
+
+def wq_version() -> int:
+    return int(lib().wq_version())
+
+
+def wq_status_string(status: int) -> str:
+    return _raw_status_string(status)
+
+
+def wq_quantize_rtn_g128(W, w_bit: int = 4, group: int = 128, zero_point: bool = True,
+                         packed=None, S=None, Z=None, stream=None):
+    """Round-to-nearest quantization of W [N, K]. INT4 asymmetric ({4, g, True}) returns
+    (packed uint8 [N, K/2], S fp16 [N, K/g], Z fp16 [N, K/g]); INT8 symmetric per channel
+    ({8, K, False}) returns (codes int8 [N, K], S fp16 [N], None)."""
+    import torch
+
+    N, K = W.shape
+    ldw = _rows(W, "W")
+    dev = W.device
+    if w_bit == 4:
+        packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev) if packed is None else packed
+        G = K // group if group else 1
+        S = torch.empty((N, G), dtype=torch.float16, device=dev) if S is None else S
+        Z = torch.empty((N, G), dtype=torch.float16, device=dev) if Z is None else Z
+    else:
+        packed = torch.empty((N, K), dtype=torch.int8, device=dev) if packed is None else packed
+        S = torch.empty((N,), dtype=torch.float16, device=dev) if S is None else S
+    p = _QParams(w_bit, group, 1 if zero_point else 0)
+    st = lib().wq_quantize_rtn_g128(_ptr(W), _w_dtype(W), N, K, ldw, ctypes.byref(p),
+                                    _ptr(packed), _ptr(S), _ptr(Z), _stream(stream))
+    _check(st, "wq_quantize_rtn_g128")
+    return packed, S, Z
+
+
+def wq_quantize_per_tensor_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().wq_quantize_per_tensor_workspace_bytes(N, K))
+
+
+def wq_quantize_rtn_per_tensor(W, workspace=None, stream=None):
+    """Per-tensor asymmetric INT4: returns (packed [N, K/2], S fp16 [1], Z fp16 [1])."""
+    import torch
+
+    N, K = W.shape
+    ldw = _rows(W, "W")
+    dev = W.device
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    S = torch.empty((1,), dtype=torch.float16, device=dev)
+    Z = torch.empty((1,), dtype=torch.float16, device=dev)
+    nbytes = wq_quantize_per_tensor_workspace_bytes(N, K)
+    if workspace is None:
+        workspace = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
+    st = lib().wq_quantize_rtn_per_tensor(_ptr(W), _w_dtype(W), N, K, ldw, _ptr(packed),
+                                          _ptr(S), _ptr(Z), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(stream))
+    _check(st, "wq_quantize_rtn_per_tensor")
+    return packed, S, Z
+
+
+def wq_pack_int4(codes, packed=None, stream=None):
+    """codes uint8 [N, K] in [0, 15] -> packed uint8 [N, K/2]."""
+    import torch
+
+    N, K = codes.shape
+    if not codes.is_contiguous():
+        raise ValueError("codes must be contiguous")
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=codes.device) if packed is None else packed
+    _check(lib().wq_pack_int4(_ptr(codes), N, K, _ptr(packed), _stream(stream)), "wq_pack_int4")
+    return packed
+
+
+def wq_dequant(packed, S, Z, group: int = 128, out_dtype=None, out=None, stream=None):
+    """W_hat = S'(q - Z) as float32 (exact) or bfloat16 [N, K]."""
+    import torch
+
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    N, K2 = packed.shape
+    K = 2 * K2
+    code = WQ_F32 if out_dtype == torch.float32 else WQ_BF16 if out_dtype == torch.bfloat16 else -1
+    out = torch.empty((N, K), dtype=out_dtype, device=packed.device) if out is None else out
+    _check(lib().wq_dequant(_ptr(packed), _ptr(S), _ptr(Z), N, K, group, _ptr(out), code,
+                            _stream(stream)), "wq_dequant")
+    return out
+
+
+def wq_w4a16_gemm(X, packed, S, Z, group: int = 128, Y=None, stream=None):
+    """Y [M, N] bf16 = X [M, K] bf16 @ W_hat^T, fp32 accumulation."""
+    import torch
+
+    M, K = X.shape
+    N = packed.shape[0]
+    ldx = _rows(X, "X")
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device) if Y is None else Y
+    ldy = _rows(Y, "Y")
+    _check(lib().wq_w4a16_gemm(_ptr(X), M, ldx, _ptr(packed), _ptr(S), _ptr(Z), N, K, group,
+                               _ptr(Y), ldy, _stream(stream)), "wq_w4a16_gemm")
+    return Y
+
+
+def wq_w8a16_gemm(X, codes, S, Y=None, stream=None):
+    """Y [M, N] bf16 = X [M, K] bf16 @ (s' q)^T with INT8 per-channel weights."""
+    import torch
+
+    M, K = X.shape
+    N = codes.shape[0]
+    ldx = _rows(X, "X")
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device) if Y is None else Y
+    ldy = _rows(Y, "Y")
+    _check(lib().wq_w8a16_gemm(_ptr(X), M, ldx, _ptr(codes), _ptr(S), N, K, _ptr(Y), ldy,
+                               _stream(stream)), "wq_w8a16_gemm")
+    return Y
+
+
+def wq_get_status(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status word."""
+    return int(lib().wq_get_status(_stream(stream)))

@@ -1,0 +1,229 @@
+// C ABI of libwq (declared in include/wq.h): argument validation, kernel choice by shape,
+// the device status word. No device memory is allocated here.
+#include <mutex>
+
+#include "../../include/wq.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_gemm.h"
+
+namespace {
+
+__device__ unsigned g_wq_status;  // per-device status word (bits wq::kSt*)
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool ready = false;
+  bool ok = false;
+  int sms = 0;
+  unsigned* status = nullptr;  // device address of g_wq_status on that device
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Current device's cached info (SM count, status-word address); nullptr if unusable.
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    d.ready = true;
+    int major = 0, minor = 0;
+    void* addr = nullptr;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        major == 10 && minor == 0 && cudaGetSymbolAddress(&addr, g_wq_status) == cudaSuccess) {
+      d.status = static_cast<unsigned*>(addr);
+      d.ok = true;
+    }
+  }
+  return d.ok ? &d : nullptr;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+wq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
+
+bool fits_int(int64_t v) { return v >= 0 && v <= 0x7fffffffLL; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t wq_version(void) { return WQ_VERSION; }
+
+const char* wq_status_string(wq_status s) {
+  switch (s) {
+    case WQ_OK: return "ok";
+    case WQ_ERR_NULL: return "a required pointer is NULL";
+    case WQ_ERR_SHAPE: return "invalid sizes (N, K, M, group or leading dimension)";
+    case WQ_ERR_ALIGN: return "pointer or leading dimension not 16-byte aligned";
+    case WQ_ERR_DTYPE: return "dtype not supported by this call";
+    case WQ_ERR_UNSUPPORTED: return "parameter combination not supported";
+    case WQ_ERR_CUDA: return "CUDA runtime error";
+    case WQ_ERR_NONFINITE: return "non-finite weight or scale overflow";
+    case WQ_ERR_TIMEOUT: return "device wait timed out";
+    case WQ_ERR_RANGE: return "code out of range [0, 15]";
+    case WQ_ERR_NODEVICE: return "no usable sm_100 CUDA device";
+  }
+  return "unknown status";
+}
+
+wq_status wq_quantize_rtn_g128(const void* W, wq_dtype w_dtype, int64_t N, int64_t K,
+                               int64_t ldw, const wq_qparams* params, uint8_t* packed,
+                               uint16_t* S, uint16_t* Z, void* stream) {
+  const wq_qparams p = params ? *params : wq_qparams{4, 128, 1};
+  if (N < 0 || K < 0) return WQ_ERR_SHAPE;
+  if (w_dtype != WQ_F32 && w_dtype != WQ_BF16) return WQ_ERR_DTYPE;
+  const bool int4 = p.w_bit == 4 && p.zero_point == 1;
+  const bool int8 = p.w_bit == 8 && p.zero_point == 0;
+  if (!int4 && !int8) return WQ_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return WQ_OK;
+  if (!W || !packed || !S || (int4 && !Z)) return WQ_ERR_NULL;
+  if (int8 && Z) return WQ_ERR_UNSUPPORTED;
+  if (!fits_int(N) || !fits_int(K) || K % 32 != 0 || ldw < K) return WQ_ERR_SHAPE;
+  if (int4 && (p.group < 32 || p.group % 32 != 0 || K % p.group != 0)) return WQ_ERR_SHAPE;
+  if (int8 && p.group != K) return WQ_ERR_UNSUPPORTED;
+  const size_t es = w_dtype == WQ_F32 ? 4 : 2;
+  if (!aligned(W, 16) || (ldw * es) % 16 != 0 || !aligned(packed, 16) || !aligned(S, 2) ||
+      (Z && !aligned(Z, 2)))
+    return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = w_dtype == WQ_BF16;
+  if (int4)
+    return from_cuda(wq::launch_quant_asym(W, bf16, ldw, (int)N, (int)K, p.group, packed, S, Z,
+                                           d->status, d->sms, st));
+  return from_cuda(wq::launch_quant_sym_int8(W, bf16, ldw, (int)N, (int)K,
+                                             reinterpret_cast<int8_t*>(packed), S, d->status,
+                                             d->sms, st));
+}
+
+size_t wq_quantize_per_tensor_workspace_bytes(int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  const DeviceInfo* d = device_info();
+  const int sms = d ? d->sms : 148;
+  return static_cast<size_t>(wq::per_tensor_parts(sms)) * sizeof(float2);
+}
+
+wq_status wq_quantize_rtn_per_tensor(const void* W, wq_dtype w_dtype, int64_t N, int64_t K,
+                                     int64_t ldw, uint8_t* packed, uint16_t* S, uint16_t* Z,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (N < 0 || K < 0) return WQ_ERR_SHAPE;
+  if (w_dtype != WQ_F32 && w_dtype != WQ_BF16) return WQ_ERR_DTYPE;
+  if (N == 0 || K == 0) return WQ_OK;
+  if (!W || !packed || !S || !Z || !workspace) return WQ_ERR_NULL;
+  if (!fits_int(N) || !fits_int(K) || K % 32 != 0 || ldw < K) return WQ_ERR_SHAPE;
+  const size_t es = w_dtype == WQ_F32 ? 4 : 2;
+  if (!aligned(W, 16) || (ldw * es) % 16 != 0 || !aligned(packed, 16) || !aligned(S, 2) ||
+      !aligned(Z, 2) || !aligned(workspace, 16))
+    return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  const int nparts = wq::per_tensor_parts(d->sms);
+  if (workspace_bytes < static_cast<size_t>(nparts) * sizeof(float2)) return WQ_ERR_SHAPE;
+  return from_cuda(wq::launch_quant_per_tensor(
+      W, w_dtype == WQ_BF16, ldw, (int)N, (int)K, packed, S, Z, static_cast<float2*>(workspace),
+      nparts, d->status, static_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_pack_int4(const uint8_t* codes, int64_t N, int64_t K, uint8_t* packed,
+                       void* stream) {
+  if (N < 0 || K < 0) return WQ_ERR_SHAPE;
+  if (N == 0 || K == 0) return WQ_OK;
+  if (!codes || !packed) return WQ_ERR_NULL;
+  if (K % 32 != 0) return WQ_ERR_SHAPE;
+  if (!aligned(codes, 16) || !aligned(packed, 16)) return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  return from_cuda(wq::launch_pack_int4(codes, N, K, packed, d->status, d->sms,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z, int64_t N,
+                     int64_t K, int32_t group, void* out, wq_dtype out_dtype, void* stream) {
+  if (N < 0 || K < 0) return WQ_ERR_SHAPE;
+  if (out_dtype != WQ_F32 && out_dtype != WQ_BF16) return WQ_ERR_DTYPE;
+  if (N == 0 || K == 0) return WQ_OK;
+  if (!packed || !S || !Z || !out) return WQ_ERR_NULL;
+  if (!fits_int(K) || K % 32 != 0) return WQ_ERR_SHAPE;
+  if (group != 0 && (group < 32 || group % 32 != 0 || K % group != 0)) return WQ_ERR_SHAPE;
+  if (!aligned(packed, 16) || !aligned(out, 16) || !aligned(S, 2) || !aligned(Z, 2))
+    return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  const int g = group ? group : (int)K;
+  const int sz_row = group ? (int)(K / group) : 0;
+  return from_cuda(wq::launch_dequant(packed, S, Z, N, (int)K, g, sz_row, out,
+                                      out_dtype == WQ_BF16, d->sms,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* packed,
+                        const uint16_t* S, const uint16_t* Z, int64_t N, int64_t K,
+                        int32_t group, uint16_t* Y, int64_t ldy, void* stream) {
+  if (M < 0 || N < 0 || K <= 0) return WQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (!X || !packed || !S || !Z || !Y) return WQ_ERR_NULL;
+  if (!fits_int(M) || !fits_int(N) || !fits_int(K) || K % 32 != 0 || ldx < K || ldy < N)
+    return WQ_ERR_SHAPE;
+  if (group != 0 && (group < 32 || group % 32 != 0 || K % group != 0)) return WQ_ERR_SHAPE;
+  if (!aligned(X, 16) || ldx % 8 != 0 || !aligned(packed, 16) || !aligned(S, 2) ||
+      !aligned(Z, 2) || !aligned(Y, 2))
+    return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int g = group ? group : (int)K;
+  const int sz_row = group ? (int)(K / group) : 0;
+  if (M <= 8 && (M > 1 || K <= wq::gemv_max_k())) {
+    wq::GemvArgs a{X, ldx, packed, S, Z, (int)M, (int)N, (int)K, g, sz_row, Y, ldy};
+    return from_cuda(wq::launch_gemv_w4a16(a, st));
+  }
+  wq::TcGemmArgs a{X, ldx, packed, S, Z, nullptr, (int)M, (int)N, (int)K, g, sz_row, Y, ldy};
+  return wq::launch_tc_gemm(a, d->sms, d->status, st);
+}
+
+wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t* codes,
+                        const uint16_t* S, int64_t N, int64_t K, uint16_t* Y, int64_t ldy,
+                        void* stream) {
+  if (M < 0 || N < 0 || K <= 0) return WQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (!X || !codes || !S || !Y) return WQ_ERR_NULL;
+  if (!fits_int(M) || !fits_int(N) || !fits_int(K) || K % 32 != 0 || ldx < K || ldy < N)
+    return WQ_ERR_SHAPE;
+  if (!aligned(X, 16) || ldx % 8 != 0 || !aligned(codes, 16) || !aligned(S, 2) ||
+      !aligned(Y, 2))
+    return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M <= 8) {
+    wq::Gemv8Args a{X, ldx, codes, S, (int)M, (int)N, (int)K, Y, ldy};
+    return from_cuda(wq::launch_gemv_w8a16(a, st));
+  }
+  wq::TcGemmArgs a{X, ldx, nullptr, S, nullptr, codes, (int)M, (int)N, (int)K, (int)K, 1, Y, ldy};
+  return wq::launch_tc_gemm(a, d->sms, d->status, st);
+}
+
+wq_status wq_get_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WQ_ERR_CUDA;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_wq_status, sizeof(v)) != cudaSuccess) return WQ_ERR_CUDA;
+  if (v != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_wq_status, &zero, sizeof(zero)) != cudaSuccess) return WQ_ERR_CUDA;
+  }
+  if (v & wq::kStNonFinite) return WQ_ERR_NONFINITE;
+  if (v & wq::kStRange) return WQ_ERR_RANGE;
+  if (v & wq::kStTimeout) return WQ_ERR_TIMEOUT;
+  return WQ_OK;
+}
+
+}  // extern "C"

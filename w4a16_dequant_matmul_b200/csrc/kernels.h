@@ -1,0 +1,53 @@
+// Internal launch interface between the C ABI layer (api.cu) and the kernel files.
+// Every launcher validates nothing: api.cu checks shapes, alignment and pointers first.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wq {
+
+cudaError_t launch_quant_asym(const void* W, bool bf16, int64_t ldw, int N, int K, int group,
+                              uint8_t* packed, uint16_t* S, uint16_t* Z, unsigned* status,
+                              int sms, cudaStream_t st);
+cudaError_t launch_quant_sym_int8(const void* W, bool bf16, int64_t ldw, int N, int K,
+                                  int8_t* codes, uint16_t* S, unsigned* status, int sms,
+                                  cudaStream_t st);
+int per_tensor_parts(int sms);
+cudaError_t launch_quant_per_tensor(const void* W, bool bf16, int64_t ldw, int N, int K,
+                                    uint8_t* packed, uint16_t* S, uint16_t* Z, float2* part,
+                                    int nparts, unsigned* status, cudaStream_t st);
+
+cudaError_t launch_pack_int4(const uint8_t* codes, int64_t N, int64_t K, uint8_t* packed,
+                             unsigned* status, int sms, cudaStream_t st);
+cudaError_t launch_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z,
+                           int64_t N, int K, int group, int sz_row, void* out, bool bf16_out,
+                           int sms, cudaStream_t st);
+
+// Small-M W4A16 matmul on CUDA cores. sz_row = scales per row (K/group), 0 = per-tensor.
+struct GemvArgs {
+  const uint16_t* X;
+  int64_t ldx;
+  const uint8_t* P;
+  const uint16_t* S;
+  const uint16_t* Z;
+  int M, N, K, group, sz_row;
+  uint16_t* Y;
+  int64_t ldy;
+};
+int gemv_max_k();
+cudaError_t launch_gemv_w4a16(const GemvArgs& a, cudaStream_t st);
+
+// Small-M W8A16 (symmetric INT8 per output channel) on CUDA cores.
+struct Gemv8Args {
+  const uint16_t* X;
+  int64_t ldx;
+  const int8_t* Q;
+  const uint16_t* S;
+  int M, N, K;
+  uint16_t* Y;
+  int64_t ldy;
+};
+cudaError_t launch_gemv_w8a16(const Gemv8Args& a, cudaStream_t st);
+
+}  // namespace wq
