@@ -1,0 +1,497 @@
+"""Benchmark of the W4A16 decode path on B200 (one JSON line on rank 0).
+
+Workload (one "step"): one decode token through three Llama-2-7B-class projection shapes,
+W4A16 g=128 (INT4 codes, binary16 S and Z per 128 weights), X bf16 1 x K:
+    4096 x 4096, 11008 x 4096, 4096 x 11008     (W: N x K, ~N(0, 0.02))
+i.e. three wq_w4a16_gemm calls at M = 1. The metric is HBM throughput of the GEMV in GB/s
+of algorithmic bytes (N*K/2 packed + 4*N*K/128 for S and Z + 2K for x + 2N for y).
+Weights cycle through rotating copies totalling more than 3x the L2 cache, so every
+launch streams its weights from HBM. Timing: CUDA graphs of the steps, CUDA events on the
+capturing stream, barrier + synchronize on both sides, max over ranks.
+
+Also reported (outside the timed step): M = 4 and 16 on the same shapes, the quantizer
+over the 70B-class weights (28672 x 8192, 8192 x 28672), the prefill GEMM
+(2048 x 4096 x 11008) when the tensor-core path is available, the oracle on the host
+cores (cpu_baseline) and the end-to-end rate through host buffers (e2e).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import wq_inputs  # noqa: E402
+
+METRIC = "W4A16 GEMV HBM GB/s (% of peak) at M=1; prefill TFLOP/s (% BF16 peak)"
+UNIT = "GB/s"
+SHAPES = wq_inputs.SHAPES_7B
+WORKLOAD = ("7B-class decode GEMV, M=1, W4A16 g128 asymmetric INT4 (fp16 S, Z), "
+            "shapes 4096x4096, 11008x4096, 4096x11008, X bf16 ~N(0,1), W ~N(0,0.02)")
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def gemv_bytes(M, N, K, group=128):
+    """Algorithmic bytes of one W4A16 matmul: packed codes, S and Z, X and Y."""
+    return N * K // 2 + 4 * N * (K // group) + 2 * M * K + 2 * M * N
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+class OracleGemv:
+    """The oracle's decode GEMV (fp64 numpy: unpack, dequantize, multiply) on a sample of
+    rows of each shape. Inputs are quantized by the oracle once, outside any timing."""
+
+    def __init__(self, shapes, rows_per_shape):
+        import oracle
+
+        self.oracle = oracle
+        self.work = []
+        for (N, K) in shapes:
+            n = min(rows_per_shape, N)
+            Wb = wq_inputs.weight_bf16(n, K, 0.02)
+            codes, S, Z = oracle.quantize_rtn_asym(wq_inputs.bf16_bits_to_f64(Wb), 128)
+            X = wq_inputs.bf16_bits_to_f64(wq_inputs.act_bf16(1, K))
+            self.work.append((oracle.pack_int4(codes), S, Z, X, n, K))
+        self.bytes = sum(gemv_bytes(1, n, K) for (_, _, _, _, n, K) in self.work)
+
+    def run(self):
+        """One pass over the sample; returns seconds."""
+        o = self.oracle
+        t0 = time.perf_counter()
+        for packed, S, Z, X, n, K in self.work:
+            Y = o.w4a16_matmul(X, o.unpack_int4(packed), S, Z, 128, "exact")
+            assert Y.shape == (1, n)
+        return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(target_s=10.0, rows=1024):
+    """Oracle GB/s on a bounded sample: `rows` rows of each shape, passes until ~target_s."""
+    og = OracleGemv(SHAPES, rows)
+    og.run()
+    tt, passes = 0.0, 0
+    while tt < target_s:
+        tt += og.run()
+        passes += 1
+    return {"value": round(og.bytes * passes / tt / 1e9, 4), "unit": UNIT,
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} rows of each of the 3 shapes at M=1 (unpack + dequant + fp64 "
+                      f"matmul), {passes} passes in {tt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = 256
+    og = OracleGemv(SHAPES, rows)
+    for _ in range(args.warmup):
+        og.run()
+    total = sum(og.run() for _ in range(args.steps))
+    value = og.bytes * args.steps / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD + f" (CPU oracle, {rows} sampled rows per shape per step)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": f"{rows} rows of each of the 3 shapes per step"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------- GPU bench
+
+def graph_time_us(fn, reps, warm=3):
+    """Per-call microseconds of `fn` captured `reps` times in one CUDA graph."""
+    import torch
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(warm):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = math.inf
+    for _ in range(3):
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1) * 1e3 / reps)
+    del g
+    return best
+
+
+def run_gpu(args):
+    import torch
+
+    import w4a16_dequant_matmul_b200 as wq
+
+    rank, world = dist_setup(args.gpus)
+    wq.build_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_src = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    # ---- weights: quantize once per shape on the GPU, then rotating copies > 3x L2
+    base = []
+    for (N, K) in SHAPES:
+        W = wq_inputs.weight_bf16(N, K, 0.02)
+        Wt = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).to(dev)
+        packed, S, Z = wq.wq_quantize_rtn_g128(Wt)
+        base.append((packed, S, Z))
+        del Wt
+    set_bytes = sum(p.numel() + 2 * s.numel() + 2 * z.numel() for p, s, z in base)
+    nsets = max(4, math.ceil(3 * l2 / set_bytes))
+    sets = [[(p.clone(), s.clone(), z.clone()) for (p, s, z) in base] for _ in range(nsets)]
+    X = [torch.from_numpy(wq_inputs.act_bf16(1, K).view(np.int16)).view(torch.bfloat16).to(dev)
+         for (_, K) in SHAPES]
+    Y = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for (N, _) in SHAPES]
+    step_bytes = sum(gemv_bytes(1, N, K) for (N, K) in SHAPES)
+    assert wq.wq_get_status() == 0
+
+    def step(i):
+        for j, (p, s, z) in enumerate(sets[i % nsets]):
+            wq.wq_w4a16_gemm(X[j], p, s, z, 128, Y=Y[j])
+
+    # one graph per rotating set (a step each) and one graph of all sets (nsets steps)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for i in range(nsets):
+            step(i)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g_one = []
+    for i in range(nsets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(i)
+        g_one.append(g)
+    g_all = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all):
+        for i in range(nsets):
+            step(i)
+
+    def run_steps(k, start=0):
+        i = start
+        while k - (i - start) >= nsets and (i % nsets) == 0:
+            g_all.replay()
+            i += nsets
+        while i - start < k:
+            g_one[i % nsets].replay()
+            i += 1
+
+    run_steps(max(args.warmup, 3))
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record()
+        run_steps(args.steps)
+        ev1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        dt_local = ev0.elapsed_time(ev1) * 1e-3
+        soak = 0
+        if dt_local < 1.5 and not args.no_soak:  # keep the step graphs running for the sampler
+            soak = int(args.steps * 1.5 / max(dt_local, 1e-6))
+            run_steps(soak)
+            torch.cuda.synchronize()
+    dt = ev0.elapsed_time(ev1) * 1e-3
+    dt = max_over_ranks(dt, world)
+    value = step_bytes * args.steps * world / dt / 1e9
+    achieved = step_bytes * args.steps / dt / 1e9   # per GPU: the dominant kernel's rate
+    assert wq.wq_get_status() == 0
+
+    # ---- per-shape kernel rates (graph of 4*nsets launches each)
+    per_shape = {}
+    for j, (N, K) in enumerate(SHAPES):
+        k = [0]
+
+        def one(j=j, k=k):
+            p, s, z = sets[k[0] % nsets][j]
+            k[0] += 1
+            wq.wq_w4a16_gemm(X[j], p, s, z, 128, Y=Y[j])
+        us = graph_time_us(one, 4 * nsets)
+        per_shape[f"{N}x{K}"] = {"us": round(us, 3), "GB/s": round(gemv_bytes(1, N, K) / us / 1e3, 1)}
+
+    # ---- secondary: M = 4, 16 on the same shapes
+    secondary = {}
+    for M in (4, 16):
+        tot_b, tot_us = 0, 0.0
+        for j, (N, K) in enumerate(SHAPES):
+            Xm = torch.from_numpy(wq_inputs.act_bf16(M, K).view(np.int16)).view(torch.bfloat16).to(dev)
+            Ym = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            k = [0]
+
+            def one(j=j, k=k, Xm=Xm, Ym=Ym):
+                p, s, z = sets[k[0] % nsets][j]
+                k[0] += 1
+                wq.wq_w4a16_gemm(Xm, p, s, z, 128, Y=Ym)
+            try:
+                us = graph_time_us(one, 2 * nsets)
+            except wq.WQError as e:
+                secondary[f"gemv_M{M}"] = f"unavailable: {e}"
+                break
+            tot_b += gemv_bytes(M, N, K)
+            tot_us += us
+        else:
+            secondary[f"gemv_M{M}_GB/s"] = round(tot_b / tot_us / 1e3, 1)
+
+    # ---- secondary: quantizer over the 70B-class weights
+    qres = {}
+    for (N, K) in wq_inputs.SHAPES_70B:
+        Wt = (torch.randn(N, K, device=dev) * 0.015).to(torch.bfloat16)
+        p = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        s = torch.empty((N, K // 128), dtype=torch.float16, device=dev)
+        z = torch.empty_like(s)
+        us = graph_time_us(lambda: wq.wq_quantize_rtn_g128(Wt, packed=p, S=s, Z=z), 5)
+        qb = N * K * 2 + N * K // 2 + 4 * N * (K // 128)
+        qres[f"{N}x{K}"] = {"us": round(us, 1), "GB/s": round(qb / us / 1e3, 1)}
+        del Wt, p, s, z
+    secondary["quantizer_70b"] = qres
+    assert wq.wq_get_status() == 0
+
+    # ---- secondary: prefill GEMM (tensor cores)
+    prefill = None
+    try:
+        P = wq_inputs.PREFILL
+        Wt = (torch.randn(P["N"], P["K"], device=dev) * 0.02).to(torch.bfloat16)
+        pk, s, z = wq.wq_quantize_rtn_g128(Wt)
+        Xp = torch.randn(P["M"], P["K"], device=dev).to(torch.bfloat16)
+        Yp = torch.empty((P["M"], P["N"]), dtype=torch.bfloat16, device=dev)
+        us = graph_time_us(lambda: wq.wq_w4a16_gemm(Xp, pk, s, z, 128, Y=Yp), 10)
+        tflops = 2.0 * P["M"] * P["N"] * P["K"] / us / 1e6
+        prefill = {"us": round(us, 1), "TFLOP/s": round(tflops, 1),
+                   "peak": peaks["bf16_tflops"], "frac": round(tflops / peaks["bf16_tflops"], 4),
+                   "shape": "M=2048 N=11008 K=4096"}
+        del Wt, pk, s, z, Xp, Yp
+    except Exception as e:  # the tensor-core path may be missing
+        prefill = f"unavailable: {e}"
+    secondary["prefill"] = prefill
+
+    # ---- e2e: through the public API with host buffers (pinned X in, Y out) per step
+    Xh = [x.cpu().pin_memory() for x in X]
+    Yh = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in Y]
+    Xd = [torch.empty_like(x) for x in X]
+    h2d = sum(x.numel() * 2 for x in X)
+    d2h = sum(y.numel() * 2 for y in Y)
+
+    def e2e_step(i):
+        for j, (p, s, z) in enumerate(sets[i % nsets]):
+            Xd[j].copy_(Xh[j], non_blocking=True)
+            wq.wq_w4a16_gemm(Xd[j], p, s, z, 128, Y=Y[j])
+            Yh[j].copy_(Y[j], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for i in range(3):
+        e2e_step(i)
+    barrier(world)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        e2e_step(i)
+    t_e2e = max_over_ranks(time.perf_counter() - t0, world)
+    e2e = {"value": round(step_bytes * args.steps * world / t_e2e / 1e9, 2), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "note": "host wall clock; per step: X H2D, 3 wq_w4a16_gemm calls via the Python "
+                   "binding, Y D2H, stream sync; weights resident (quantized once)"}
+
+    if rank == 0:
+        traffic = None
+        tf = os.path.join(ROOT, "profiles", "gemv_traffic.json")
+        if os.path.exists(tf):
+            with open(tf) as f:
+                traffic = json.load(f).get("bytes_per_step")
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": 1, "group": 128,
+                       "l2": f"inputs larger than L2: {nsets} rotating weight sets, "
+                             f"{nsets * set_bytes / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB",
+                       "bytes_per_step": step_bytes, "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                         "peak_source": peak_src, "kernel": "gemv_slices (M=1)"},
+            "per_shape": per_shape,
+            "secondary": secondary,
+            "clocks": dict(clk.summary(), **({"soak_steps_after_timed_region": soak}
+                                             if soak else {})),
+            "e2e": e2e,
+            "gpu_launches": len(SHAPES) * args.steps,
+            "cpu_baseline": cpu_baseline() if not args.no_cpu_baseline else None,
+        }
+        print(json.dumps(line), flush=True)
+    del g_one, g_all
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="libwq", choices=["libwq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-soak", action="store_true",
+                    help="no clock soak after a short timed region (for profiler runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
