@@ -102,6 +102,19 @@ wq_status wq_quantize_rtn_per_tensor(const void* W, wq_dtype w_dtype, int64_t N,
                                      uint16_t* Z, void* workspace, size_t workspace_bytes,
                                      void* stream);
 
+/* Per-tensor asymmetric INT4 like wq_quantize_rtn_per_tensor, for callers that cannot
+ * allocate device memory (no workspace argument; nothing is allocated). The pages have no
+ * counterpart: this is a deployment variant. The grid-wide min/max goes to a fixed 32 KB
+ * array inside the library (4096 (min, max) slots; 8 are used per SM, so a device with
+ * more than 512 SMs gets WQ_ERR_UNSUPPORTED). The array exists once per device for as
+ * long as the library is loaded, and all calls on a device share it, so calls that
+ * overlap on the GPU race with one another. The first call on each device looks up the
+ * array's device address; make it before any stream capture. Outputs as for
+ * wq_quantize_rtn_per_tensor. */
+wq_status wq_quantize_rtn_per_tensor_noalloc(const void* W, wq_dtype w_dtype, int64_t N,
+                                             int64_t K, int64_t ldw, uint8_t* packed,
+                                             uint16_t* S, uint16_t* Z, void* stream);
+
 /* Pack 4-bit codes two per byte (the storage of "INT4 weights + FP16 scales/zero-points",
  * "Model Quantization", section 4): codes [N, K] uint8 in [0, 15] -> packed [N, K/2].
  * A code above 15 sets WQ_ERR_RANGE in the status word. Requires K % 32 == 0. */

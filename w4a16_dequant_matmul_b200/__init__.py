@@ -25,7 +25,8 @@ from ._build import LIB_PATH, build_library  # noqa: F401  (build_library re-exp
 __all__ = [
     "WQError", "lib", "status_name",
     "wq_version", "wq_status_string", "wq_quantize_rtn_g128", "wq_quantize_rtn_per_tensor",
-    "wq_quantize_per_tensor_workspace_bytes", "wq_pack_int4", "wq_dequant", "wq_w4a16_gemm",
+    "wq_quantize_per_tensor_workspace_bytes", "wq_quantize_rtn_per_tensor_noalloc",
+    "wq_pack_int4", "wq_dequant", "wq_w4a16_gemm",
     "wq_w8a16_gemm", "wq_get_status",
     "WQ_F32", "WQ_BF16", "WQ_F16", "WQ_U8", "WQ_I8",
 ]
@@ -62,6 +63,7 @@ _SIGNATURES = {
     "wq_quantize_per_tensor_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
     "wq_quantize_rtn_per_tensor": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P,
                                           ctypes.c_size_t, _P]),
+    "wq_quantize_rtn_per_tensor_noalloc": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]),
     "wq_pack_int4": (_I32, [_P, _I64, _I64, _P, _P]),
     "wq_dequant": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _I32, _P]),
     "wq_w4a16_gemm": (_I32, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I32, _P, _I64, _P]),
@@ -184,6 +186,24 @@ def wq_quantize_rtn_per_tensor(W, workspace=None, stream=None):
                                           workspace.numel() * workspace.element_size(),
                                           _stream(stream))
     _check(st, "wq_quantize_rtn_per_tensor")
+    return packed, S, Z
+
+
+def wq_quantize_rtn_per_tensor_noalloc(W, stream=None):
+    """Per-tensor asymmetric INT4 without a workspace (for callers that cannot allocate
+    device memory); the library's own fixed scratch array is used. Returns
+    (packed [N, K/2], S fp16 [1], Z fp16 [1]). Output tensors are allocated here by torch
+    only for convenience; C callers pass their own."""
+    import torch
+
+    N, K = W.shape
+    ldw = _rows(W, "W")
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    S = torch.empty((1,), dtype=torch.float16, device=W.device)
+    Z = torch.empty((1,), dtype=torch.float16, device=W.device)
+    st = lib().wq_quantize_rtn_per_tensor_noalloc(_ptr(W), _w_dtype(W), N, K, ldw, _ptr(packed),
+                                                  _ptr(S), _ptr(Z), _stream(stream))
+    _check(st, "wq_quantize_rtn_per_tensor_noalloc")
     return packed, S, Z
 
 

@@ -50,6 +50,16 @@ bool fits_int(int64_t v) { return v >= 0 && v <= 0x7fffffffLL; }
 
 }  // namespace
 
+namespace wq {
+bool current_device(int* sms, unsigned** status) {
+  const DeviceInfo* d = device_info();
+  if (!d) return false;
+  *sms = d->sms;
+  *status = d->status;
+  return true;
+}
+}  // namespace wq
+
 extern "C" {
 
 int32_t wq_version(void) { return WQ_VERSION; }

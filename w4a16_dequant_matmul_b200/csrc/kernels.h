@@ -7,6 +7,10 @@
 
 namespace wq {
 
+// SM count and device address of the status word for the current device (false if there
+// is no usable sm_100 device). Defined in api.cu.
+bool current_device(int* sms, unsigned** status);
+
 cudaError_t launch_quant_asym(const void* W, bool bf16, int64_t ldw, int N, int K, int group,
                               uint8_t* packed, uint16_t* S, uint16_t* Z, unsigned* status,
                               int sms, cudaStream_t st);
