@@ -191,8 +191,8 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
   const int g = group ? group : (int)K;
   const int sz_row = group ? (int)(K / group) : 0;
   if (M <= 8 && (M > 1 || K <= wq::gemv_max_k())) {
-    wq::GemvArgs a{X, ldx, packed, S, Z, (int)M, (int)N, (int)K, g, sz_row, Y, ldy};
-    return from_cuda(wq::launch_gemv_w4a16(a, st));
+    wq::GemvArgs a{X, ldx, packed, S, Z, (int)M, (int)N, (int)K, g, sz_row, Y, ldy, d->status};
+    return from_cuda(wq::launch_gemv_w4a16(a, d->sms, st));
   }
   wq::TcGemmArgs a{X, ldx, packed, S, Z, nullptr, (int)M, (int)N, (int)K, g, sz_row, Y, ldy};
   return wq::launch_tc_gemm(a, d->sms, d->status, st);

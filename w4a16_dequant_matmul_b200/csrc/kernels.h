@@ -38,9 +38,10 @@ struct GemvArgs {
   int M, N, K, group, sz_row;
   uint16_t* Y;
   int64_t ldy;
+  unsigned* status;
 };
 int gemv_max_k();
-cudaError_t launch_gemv_w4a16(const GemvArgs& a, cudaStream_t st);
+cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st);
 
 // Small-M W8A16 (symmetric INT8 per output channel) on CUDA cores.
 struct Gemv8Args {
