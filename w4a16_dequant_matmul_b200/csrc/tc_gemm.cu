@@ -1,10 +1,451 @@
-// Tensor-core W4A16 / W8A16 GEMM (placeholder until the tcgen05 kernel lands).
+// Tensor-core W4A16 / W8A16 GEMM for B200 (tcgen05 + TMEM + TMA), Y = X W_hat^T.
+// ("LLM Weight Quantization - GPTQ, AWQ, SmoothQuant, FP8 & INT4/INT8 Trade-offs",
+// "The vocabulary": 4-bit weights dequantized to 16 bits inside the kernel, 16-bit matmul;
+// the prefill "still runs 16-bit math", so this is the compute-bound half of the path.)
+//
+// Tile: 128 weight rows (MMA M) x 256 tokens (MMA N), K in stages of 64. The weight tile is
+// the MMA's A operand so that a dequantized tile feeds 256 tokens at once. Per CTA
+// (persistent, one per SM), warp roles:
+//   warp 0      TMA producer: X tiles [256 tokens x 64 k] bf16, 128-byte swizzle, into the
+//               stage ring (completes on the stage's "full" mbarrier).
+//   warp 1      allocates TMEM (512 columns = two 128 x 256 fp32 accumulators); lane 0
+//               issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32), 4 per stage, and
+//               commits each stage to its "empty" barrier and each tile to "acc_full".
+//   warps 2-5   dequantizers: thread r owns weight row r of the tile; it loads its 32
+//               packed bytes (64 codes) per stage, forms W_hat = S'(q - Z) exactly in fp32
+//               (one byte-permute and one FMA per weight), rounds to bf16 and writes the
+//               row into the A tile in the canonical K-major 128-byte-swizzled layout.
+//   warps 6-9   epilogue: tcgen05.ld the accumulator (32 rows per warp, its TMEM lane
+//               quarter), round to bf16, stage [256 tokens x 128 rows] in shared memory
+//               and write it to Y with one TMA store per tile.
+// Every mbarrier wait is bounded (2 s): on a timeout the kernel records kStTimeout and all
+// roles leave their loops, drain outstanding work with bounded waits, free TMEM and exit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "ptx.cuh"
 #include "tc_gemm.h"
 
 namespace wq {
+namespace {
 
-wq_status launch_tc_gemm(const TcGemmArgs&, int, unsigned*, cudaStream_t) {
-  return WQ_ERR_UNSUPPORTED;
+constexpr int kRows = 128;     // weight rows per tile (MMA M)
+constexpr int kToks = 256;     // tokens per tile (MMA N)
+constexpr int kBK = 64;        // k per stage (one 128-byte swizzle atom of bf16)
+constexpr int kStages = 3;
+constexpr int kABytes = kRows * kBK * 2;    // 16 KB
+constexpr int kBBytes = kToks * kBK * 2;    // 32 KB
+constexpr int kEpiBytes = kToks * kRows * 2;  // 64 KB
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kLimitNs = 2000000000ull;
+
+struct Smem {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  volatile int abort;
+};
+constexpr size_t kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kEpiBytes + sizeof(Smem);
+
+// --- tcgen05 / TMA wrappers --------------------------------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets its lane's columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x,
+                                             int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::
+                   "l"(map),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of 128 bytes
+// in 1024-byte atoms of 8 rows (stride between atoms 1024 B), sm100 descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(const void* p) {
+  const uint64_t addr = smem_u32(p);
+  return ((addr & 0x3FFFFull) >> 4) | (1ull << 16) | ((1024ull >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, M = 128, N = 256.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kToks >> 3) << 17) |
+                            ((kRows >> 4) << 24);
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Smem* sm,
+                                              unsigned* status) {
+  if (mbar_wait_bounded(bar, parity, kLimitNs)) return true;
+  set_status(status, kStTimeout);
+  atomicExch(const_cast<int*>(&sm->abort), 1);
+  return false;
+}
+
+// Dequantize 64 codes of one row (32 packed bytes, or 64 int8 bytes) into 8 chunks of 8
+// bf16 values and store them into the swizzled A tile row.
+__device__ __forceinline__ void store_row_chunk(uint8_t* tile, int r, int c, const float* w) {
+  uint4 v;
+  v.x = pack_bf16x2(w[0], w[1]);
+  v.y = pack_bf16x2(w[2], w[3]);
+  v.z = pack_bf16x2(w[4], w[5]);
+  v.w = pack_bf16x2(w[6], w[7]);
+  *reinterpret_cast<uint4*>(tile + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = v;
+}
+
+// Eight codes of a 32-bit word (nibble i = code of k = i) -> S'(q - Z), exact in fp32:
+// f = 0.5 + q/256 from one byte-permute; 256 S' f - S'(128 + Z) = S'(q - Z).
+__device__ __forceinline__ void dq8_int4(uint32_t word, float s256, float c0, float* w) {
+  const uint32_t lo = word & 0x0F0F0F0Fu;
+  const uint32_t hi = (word >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t sel = 0x7044u | (static_cast<uint32_t>(j) << 8);
+    w[2 * j] = fmaf(__uint_as_float(__byte_perm(lo, 0x3F000000u, sel)), s256, c0);
+    w[2 * j + 1] = fmaf(__uint_as_float(__byte_perm(hi, 0x3F000000u, sel)), s256, c0);
+  }
+}
+
+// Four int8 codes of a word -> s' q, exact in fp32 (q from 2^23 + (b ^ 0x80) - 2^23 - 128).
+__device__ __forceinline__ void dq4_int8(uint32_t word, float s, float* w) {
+  const uint32_t u = word ^ 0x80808080u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float q = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440u | j)) - 8388736.0f;
+    w[j] = s * q;
+  }
+}
+
+template <bool kInt8>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+               const uint8_t* __restrict__ P, const int8_t* __restrict__ Q8,
+               const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int M, int N,
+               int K, int group, int sz_row, unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* tileA = base;                              // [kStages][kABytes]
+  uint8_t* tileB = base + kStages * kABytes;          // [kStages][kBBytes]
+  uint8_t* epi = tileB + kStages * kBBytes;           // [kToks][kRows] bf16
+  Smem* sm = reinterpret_cast<Smem*>(epi + kEpiBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tiles = (N + kRows - 1) / kRows;
+  const int m_tiles = (M + kToks - 1) / kToks;
+  const int tiles = n_tiles * m_tiles;
+  const int KB = K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm->full[s], 1 + 4);  // TMA arrive.expect_tx + 4 dequant warps
+      mbar_init(&sm->empty[s], 1);     // tcgen05.commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm->acc_full[b], 1);
+      mbar_init(&sm->acc_empty[b], 4);
+    }
+    mbar_init(&sm->done, 1);
+    sm->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x) {
+        const int mt = t % m_tiles;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t u = it / kStages;
+          if (u > 0 && !wait_or_abort(&sm->empty[s], (u - 1) & 1u, sm, status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm->full[s], kBBytes);
+          tma_load_2d(tileB + s * kBBytes, &tmX, kb * kBK, mt * kToks, &sm->full[s]);
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, j = 0;
+      for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x, ++j) {
+        const int b = j & 1;
+        if (j >= 2 && !wait_or_abort(&sm->acc_empty[b], ((j >> 1) - 1) & 1u, sm, status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + b * kToks;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!wait_or_abort(&sm->full[s], (it / kStages) & 1u, sm, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* a = tileA + s * kABytes;
+          const uint8_t* bt = tileB + s * kBBytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            tc_mma(d, sw128_desc(a + 32 * k), sw128_desc(bt + 32 * k), kIdesc,
+                   (kb | k) != 0 ? 1u : 0u);
+          tc_commit(&sm->empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&sm->acc_full[b]);
+      }
+      // all issued MMAs have completed once this commit arrives
+      tc_commit(&sm->done);
+      if (!mbar_wait_bounded(&sm->done, 0, kLimitNs)) set_status(status, kStTimeout);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ dequantizers
+    const int r = threadIdx.x - 64;  // 0..127: weight row within the tile
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x) {
+      const int nt = t / m_tiles;
+      const int n = nt * kRows + r;
+      const bool valid = n < N;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % kStages;
+        const uint32_t u = it / kStages;
+        // global loads first (they do not touch the stage), then wait for the slot
+        float w[64];
+        if (!kInt8) {
+          uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
+          float s256[2] = {0.0f, 0.0f}, c0[2] = {0.0f, 0.0f};
+          if (valid) {
+            const uint8_t* src = P + static_cast<int64_t>(n) * (K / 2) + kb * (kBK / 2);
+            p0 = ld_nc_u4(src);
+            p1 = ld_nc_u4(src + 16);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int64_t gi =
+                  static_cast<int64_t>(n) * sz_row + (sz_row ? (kb * kBK + 32 * h) / group : 0);
+              const float sv = f16_bits_to_f32(ld_nc_u16(S + gi));
+              const float zv = f16_bits_to_f32(ld_nc_u16(Zp + gi));
+              s256[h] = 256.0f * sv;
+              c0[h] = -sv * (128.0f + zv);
+            }
+          }
+          const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) dq8_int4(words[q], s256[q >> 2], c0[q >> 2], w + 8 * q);
+        } else {
+          uint4 v[4] = {};
+          float sv = 0.0f;
+          if (valid) {
+            const int8_t* src = Q8 + static_cast<int64_t>(n) * K + kb * kBK;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[q] = ld_nc_u4(src + 16 * q);
+            sv = f16_bits_to_f32(ld_nc_u16(S + n));
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            dq4_int8(v[q].x, sv, w + 16 * q);
+            dq4_int8(v[q].y, sv, w + 16 * q + 4);
+            dq4_int8(v[q].z, sv, w + 16 * q + 8);
+            dq4_int8(v[q].w, sv, w + 16 * q + 12);
+          }
+        }
+        if (u > 0 && !wait_or_abort(&sm->empty[s], (u - 1) & 1u, sm, status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* tile = tileA + s * kABytes;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) store_row_chunk(tile, r, c, w + 8 * c);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->full[s]);
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ---------------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 (this warp's access window)
+    const int row = quarter * 32 + lane;
+    const bool leader = (threadIdx.x == 192);
+    uint32_t j = 0;
+    for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x, ++j) {
+      const int nt = t / m_tiles, mt = t % m_tiles;
+      const int b = j & 1;
+      if (!wait_or_abort(&sm->acc_full[b], (j >> 1) & 1u, sm, status)) break;
+      tc_fence_after();
+      if (leader) bulk_wait_read0();  // the previous tile's store has read the staging buffer
+      named_barrier(2, 128);
+      uint16_t* st = reinterpret_cast<uint16_t*>(epi);
+      for (int c = 0; c < kToks / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * kToks + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
+          st[(c * 32 + i) * kRows + row] = *reinterpret_cast<uint16_t*>(&h);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
+      fence_async_smem();
+      named_barrier(2, 128);
+      if (leader) {
+        tma_store_2d(&tmY, epi, nt * kRows, mt * kToks);
+        bulk_commit();
+      }
+    }
+    if (leader) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// --- host: tensor maps -----------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+wq_status launch_tc_gemm(const TcGemmArgs& a, int sms, unsigned* status, cudaStream_t st) {
+  const bool int8 = a.Q8 != nullptr;
+  if (a.K % kBK != 0) return WQ_ERR_SHAPE;
+  if (!int8 && a.sz_row && a.group % 32 != 0) return WQ_ERR_SHAPE;
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!al16(a.X) || !al16(a.Y) || a.ldx % 8 != 0 || a.ldy % 8 != 0) return WQ_ERR_ALIGN;
+  CUtensorMap mx, my;
+  if (!make_map(&mx, a.X, a.K, a.M, a.ldx * 2, kBK, kToks, true)) return WQ_ERR_CUDA;
+  if (!make_map(&my, a.Y, a.N, a.M, a.ldy * 2, kRows, kToks, false)) return WQ_ERR_CUDA;
+  auto kern = int8 ? tc_gemm_kernel<true> : tc_gemm_kernel<false>;
+  static bool attr[2] = {false, false};
+  if (!attr[int8]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return WQ_ERR_CUDA;
+    attr[int8] = true;
+  }
+  const int tiles = ((a.N + kRows - 1) / kRows) * ((a.M + kToks - 1) / kToks);
+  const int grid = tiles < sms ? tiles : sms;
+  kern<<<grid, kThreads, kSmemBytes, st>>>(mx, my, a.P, a.Q8, a.S, a.Z, a.M, a.N, a.K, a.group,
+                                           a.sz_row, status);
+  return cudaGetLastError() == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
 }  // namespace wq
