@@ -267,17 +267,16 @@ gemv_m1_bulk(const uint16_t* __restrict__ X, const uint8_t* __restrict__ P,
       set_status(status, kStTimeout);
       return;
     }
-    const uint8_t* base = smem + static_cast<size_t>(st) * stage_bytes;
-    const uint16_t* sS = reinterpret_cast<const uint16_t*>(base + pbytes);
-    const uint16_t* sZ = sS + RB * G;
+    const uint32_t base = smem_u32(smem) + st * stage_bytes;
+    const uint32_t sS = base + pbytes;
+    const uint32_t sZ = sS + sbytes;
     float acc[RW];
 #pragma unroll
     for (int rr = 0; rr < RW; ++rr) {
       const int r = wr + rr * WR;
-      const uint4 pk = kact ? *reinterpret_cast<const uint4*>(base + r * (K / 2) + k0 / 2)
-                            : make_uint4(0, 0, 0, 0);
-      const float sv = f16_bits_to_f32(sS[r * G + gik]);
-      const float zv = f16_bits_to_f32(sZ[r * G + gik]);
+      const uint4 pk = kact ? lds128(base + r * (K / 2) + k0 / 2) : make_uint4(0, 0, 0, 0);
+      const float sv = f16_bits_to_f32(lds16(sS + (r * G + gik) * 2));
+      const float zv = f16_bits_to_f32(lds16(sZ + (r * G + gik) * 2));
       float2 a2 = make_float2(0.0f, 0.0f);
       const uint32_t ws[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll

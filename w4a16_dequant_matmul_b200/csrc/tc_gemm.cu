@@ -11,11 +11,12 @@
 //   warp 1      allocates TMEM (512 columns = two 128 x 256 fp32 accumulators); lane 0
 //               issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32), 4 per stage, and
 //               commits each stage to its "empty" barrier and each tile to "acc_full".
-//   warps 2-5   dequantizers: thread r owns weight row r of the tile; it loads its 32
-//               packed bytes (64 codes) per stage, forms W_hat = S'(q - Z) exactly in fp32
-//               (one byte-permute and one FMA per weight), rounds to bf16 and writes the
-//               row into the A tile in the canonical K-major 128-byte-swizzled layout.
-//   warps 6-9   epilogue: tcgen05.ld the accumulator (32 rows per warp, its TMEM lane
+//   warps 2-9   dequantizers: thread (h, r) owns half h of weight row r of the stage; it
+//               keeps the packed bytes and S', Z of the next two stages in flight, forms
+//               W_hat = S'(q - Z) exactly in fp32 (one byte-permute per weight, packed
+//               fp32x2 FMAs), rounds to bf16 and writes its 32 values into the A tile in
+//               the canonical K-major 128-byte-swizzled layout.
+//   warps 10-13 epilogue: tcgen05.ld the accumulator (32 rows per warp, its TMEM lane
 //               quarter), round to bf16, stage [256 tokens x 128 rows] in shared memory
 //               and write it to Y with one TMA store per tile.
 // Every mbarrier wait is bounded (2 s): on a timeout the kernel records kStTimeout and all
@@ -35,24 +36,36 @@ namespace {
 constexpr int kRows = 128;     // weight rows per tile (MMA M)
 constexpr int kToks = 256;     // tokens per tile (MMA N)
 constexpr int kBK = 64;        // k per stage (one 128-byte swizzle atom of bf16)
-constexpr int kStages = 3;
-constexpr int kABytes = kRows * kBK * 2;    // 16 KB
-constexpr int kBBytes = kToks * kBK * 2;    // 32 KB
-constexpr int kEpiBytes = kToks * kRows * 2;  // 64 KB
-constexpr int kThreads = 320;
+constexpr int kABytes = kRows * kBK * 2;    // 16 KB: dequantized bf16 weight tile
+constexpr int kBBytes = kToks * kBK * 2;    // 32 KB: X tile
+constexpr int kEpiToks = 64;                // tokens per epilogue store
+constexpr int kEpiBytes = kEpiToks * kRows * 2;  // 16 KB
+// Stage ring depth and raw-code bytes per stage: INT4 keeps 32 B/row, INT8 64 B/row.
+template <bool kInt8> struct Cfg {
+  static constexpr int kRBytes = kRows * (kInt8 ? kBK : kBK / 2);
+  static constexpr int kStages = kInt8 ? 3 : 4;
+};
+constexpr int kMaxStages = 4;
+constexpr int kThreads = 448;  // 14 warps: TMA, MMA, 8 dequant, 4 epilogue
+constexpr int kDqWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kLimitNs = 2000000000ull;
 
 struct Smem {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t raw_full[kMaxStages];  // TMA: X tile + raw weight codes landed (tx bytes)
+  uint64_t full[kMaxStages];      // dequant warps: bf16 weight tile written
+  uint64_t empty[kMaxStages];     // tcgen05.commit: the stage's MMAs are done
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t done;
   uint32_t tmem_base;
   volatile int abort;
 };
-constexpr size_t kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kEpiBytes + sizeof(Smem);
+template <bool kInt8>
+constexpr size_t smem_bytes() {
+  return 1024 + Cfg<kInt8>::kStages * (kABytes + kBBytes + Cfg<kInt8>::kRBytes) + kEpiBytes +
+         sizeof(Smem);
+}
 
 // --- tcgen05 / TMA wrappers --------------------------------------------------------
 
@@ -155,13 +168,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm
 
 // Dequantize 64 codes of one row (32 packed bytes, or 64 int8 bytes) into 8 chunks of 8
 // bf16 values and store them into the swizzled A tile row.
-__device__ __forceinline__ void store_row_chunk(uint8_t* tile, int r, int c, const float* w) {
+__device__ __forceinline__ void store_row_chunk(uint32_t tile, int r, int c, const float* w) {
   uint4 v;
   v.x = pack_bf16x2(w[0], w[1]);
   v.y = pack_bf16x2(w[2], w[3]);
   v.z = pack_bf16x2(w[4], w[5]);
   v.w = pack_bf16x2(w[6], w[7]);
-  *reinterpret_cast<uint4*>(tile + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = v;
+  sts128(tile + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4), v);
 }
 
 // Eight codes of a 32-bit word (nibble i = code of k = i) -> S'(q - Z), exact in fp32:
@@ -169,11 +182,15 @@ __device__ __forceinline__ void store_row_chunk(uint8_t* tile, int r, int c, con
 __device__ __forceinline__ void dq8_int4(uint32_t word, float s256, float c0, float* w) {
   const uint32_t lo = word & 0x0F0F0F0Fu;
   const uint32_t hi = (word >> 4) & 0x0F0F0F0Fu;
+  const float2 a2 = make_float2(s256, s256), c2 = make_float2(c0, c0);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t sel = 0x7044u | (static_cast<uint32_t>(j) << 8);
-    w[2 * j] = fmaf(__uint_as_float(__byte_perm(lo, 0x3F000000u, sel)), s256, c0);
-    w[2 * j + 1] = fmaf(__uint_as_float(__byte_perm(hi, 0x3F000000u, sel)), s256, c0);
+    const float2 f = make_float2(__uint_as_float(__byte_perm(lo, 0x3F000000u, sel)),
+                                 __uint_as_float(__byte_perm(hi, 0x3F000000u, sel)));
+    const float2 v = __ffma2_rn(f, a2, c2);
+    w[2 * j] = v.x;
+    w[2 * j + 1] = v.y;
   }
 }
 
@@ -190,15 +207,19 @@ __device__ __forceinline__ void dq4_int8(uint32_t word, float s, float* w) {
 template <bool kInt8>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
-               const uint8_t* __restrict__ P, const int8_t* __restrict__ Q8,
+               const __grid_constant__ CUtensorMap tmW, const uint8_t* __restrict__ P,
+               const int8_t* __restrict__ Q8,
                const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int M, int N,
                int K, int group, int sz_row, unsigned* status) {
+  constexpr int kStages = Cfg<kInt8>::kStages;
+  constexpr int kRBytes = Cfg<kInt8>::kRBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* tileA = base;                              // [kStages][kABytes]
   uint8_t* tileB = base + kStages * kABytes;          // [kStages][kBBytes]
-  uint8_t* epi = tileB + kStages * kBBytes;           // [kToks][kRows] bf16
+  uint8_t* tileR = tileB + kStages * kBBytes;         // [kStages][kRBytes]
+  uint8_t* epi = tileR + kStages * kRBytes;           // [kEpiToks][kRows] bf16
   Smem* sm = reinterpret_cast<Smem*>(epi + kEpiBytes);
 
   const int warp = threadIdx.x >> 5;
@@ -210,7 +231,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm->full[s], 1 + 4);  // TMA arrive.expect_tx + 4 dequant warps
+      mbar_init(&sm->raw_full[s], 1);       // TMA arrive.expect_tx
+      mbar_init(&sm->full[s], kDqWarps);    // dequant warps
       mbar_init(&sm->empty[s], 1);     // tcgen05.commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -234,8 +256,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       uint32_t it = 0;
+      const uint32_t rbytes = kInt8 ? kRows * kBK : kRows * kBK / 2;
       for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x) {
-        const int mt = t % m_tiles;
+        const int nt = t / m_tiles, mt = t % m_tiles;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kStages;
@@ -244,8 +267,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&sm->full[s], kBBytes);
-          tma_load_2d(tileB + s * kBBytes, &tmX, kb * kBK, mt * kToks, &sm->full[s]);
+          mbar_arrive_expect_tx(&sm->raw_full[s], kBBytes + rbytes);
+          tma_load_2d(tileB + s * kBBytes, &tmX, kb * kBK, mt * kToks, &sm->raw_full[s]);
+          tma_load_2d(tileR + s * kRBytes, &tmW, kb * (kInt8 ? kBK : kBK / 2), nt * kRows,
+                      &sm->raw_full[s]);
         }
         if (!ok) break;
       }
@@ -262,7 +287,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kStages;
-          if (!wait_or_abort(&sm->full[s], (it / kStages) & 1u, sm, status)) {
+          if (!wait_or_abort(&sm->raw_full[s], (it / kStages) & 1u, sm, status) ||
+              !wait_or_abort(&sm->full[s], (it / kStages) & 1u, sm, status)) {
             ok = false;
             break;
           }
@@ -282,64 +308,74 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
       tc_commit(&sm->done);
       if (!mbar_wait_bounded(&sm->done, 0, kLimitNs)) set_status(status, kStTimeout);
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kDqWarps) {
     // ------------------------------------------------------------------ dequantizers
-    const int r = threadIdx.x - 64;  // 0..127: weight row within the tile
+    // Lane pairs share a weight row: thread (r, h) handles half h (32 k) of row r, so a
+    // quarter-warp reads 128 contiguous bytes of the raw tile and writes 8 distinct
+    // 16-byte slots of the swizzled A tile (both bank-conflict free).
+    const int td = threadIdx.x - 64;                  // 0..255
+    const int r = (td >> 5) * 16 + ((td & 31) >> 1);  // weight row within the tile
+    const int h = td & 1;                             // which 32-k half of the stage
+    // (tile, kb) of the iteration whose scales are fetched next, advanced incrementally
+    int f_t = blockIdx.x, f_kb = 0;
+    auto fetch = [&](float& fa, float& fc) {
+      fa = fc = 0.0f;
+      if (f_t >= tiles) return;
+      const int n = (f_t / m_tiles) * kRows + r;
+      if (n < N) {
+        if (!kInt8) {
+          const int k0 = f_kb * kBK + 32 * h;
+          const int64_t gi = static_cast<int64_t>(n) * sz_row + (sz_row ? k0 / group : 0);
+          const float sv = f16_bits_to_f32(ld_nc_u16(S + gi));
+          const float zv = f16_bits_to_f32(ld_nc_u16(Zp + gi));
+          fa = 256.0f * sv;
+          fc = -sv * (128.0f + zv);
+        } else {
+          fa = f16_bits_to_f32(ld_nc_u16(S + n));
+        }
+      }
+      if (++f_kb == KB) {
+        f_kb = 0;
+        f_t += gridDim.x;
+      }
+    };
+    float a0, c0, a1, c1;
+    fetch(a0, c0);
+    fetch(a1, c1);
+    const uint32_t tileA_s = smem_u32(tileA), tileR_s = smem_u32(tileR);
     uint32_t it = 0;
     for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x) {
-      const int nt = t / m_tiles;
-      const int n = nt * kRows + r;
-      const bool valid = n < N;
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb, ++it) {
+        const float ca = a0, cc = c0;
+        a0 = a1;
+        c0 = c1;
+        fetch(a1, c1);
         const int s = it % kStages;
         const uint32_t u = it / kStages;
-        // global loads first (they do not touch the stage), then wait for the slot
-        float w[64];
-        if (!kInt8) {
-          uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
-          float s256[2] = {0.0f, 0.0f}, c0[2] = {0.0f, 0.0f};
-          if (valid) {
-            const uint8_t* src = P + static_cast<int64_t>(n) * (K / 2) + kb * (kBK / 2);
-            p0 = ld_nc_u4(src);
-            p1 = ld_nc_u4(src + 16);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int64_t gi =
-                  static_cast<int64_t>(n) * sz_row + (sz_row ? (kb * kBK + 32 * h) / group : 0);
-              const float sv = f16_bits_to_f32(ld_nc_u16(S + gi));
-              const float zv = f16_bits_to_f32(ld_nc_u16(Zp + gi));
-              s256[h] = 256.0f * sv;
-              c0[h] = -sv * (128.0f + zv);
-            }
-          }
-          const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-          for (int q = 0; q < 8; ++q) dq8_int4(words[q], s256[q >> 2], c0[q >> 2], w + 8 * q);
-        } else {
-          uint4 v[4] = {};
-          float sv = 0.0f;
-          if (valid) {
-            const int8_t* src = Q8 + static_cast<int64_t>(n) * K + kb * kBK;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) v[q] = ld_nc_u4(src + 16 * q);
-            sv = f16_bits_to_f32(ld_nc_u16(S + n));
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            dq4_int8(v[q].x, sv, w + 16 * q);
-            dq4_int8(v[q].y, sv, w + 16 * q + 4);
-            dq4_int8(v[q].z, sv, w + 16 * q + 8);
-            dq4_int8(v[q].w, sv, w + 16 * q + 12);
-          }
-        }
-        if (u > 0 && !wait_or_abort(&sm->empty[s], (u - 1) & 1u, sm, status)) {
+        // the raw codes of this stage have landed (which also means the stage's previous
+        // MMAs are done, since the TMA for it was issued only after "empty")
+        if (!wait_or_abort(&sm->raw_full[s], u & 1u, sm, status)) {
           ok = false;
           break;
         }
-        uint8_t* tile = tileA + s * kABytes;
+        const uint32_t raw = tileR_s + s * kRBytes;
+        float w[32];
+        if (!kInt8) {
+          const uint4 p = lds128(raw + r * (kBK / 2) + 16 * h);
+          const uint32_t words[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) store_row_chunk(tile, r, c, w + 8 * c);
+          for (int q = 0; q < 4; ++q) dq8_int4(words[q], ca, cc, w + 8 * q);
+        } else {
+          const uint4 p0 = lds128(raw + r * kBK + 32 * h);
+          const uint4 p1 = lds128(raw + r * kBK + 32 * h + 16);
+          const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) dq4_int8(words[q], ca, w + 4 * q);
+        }
+        const uint32_t tile = tileA_s + s * kABytes;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) store_row_chunk(tile, r, 4 * h + c, w + 8 * c);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->full[s]);
@@ -350,34 +386,40 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     // ---------------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 (this warp's access window)
     const int row = quarter * 32 + lane;
-    const bool leader = (threadIdx.x == 192);
+    const bool leader = (threadIdx.x == 32 * (2 + kDqWarps));
     uint32_t j = 0;
     for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x, ++j) {
       const int nt = t / m_tiles, mt = t % m_tiles;
       const int b = j & 1;
       if (!wait_or_abort(&sm->acc_full[b], (j >> 1) & 1u, sm, status)) break;
       tc_fence_after();
-      if (leader) bulk_wait_read0();  // the previous tile's store has read the staging buffer
-      named_barrier(2, 128);
-      uint16_t* st = reinterpret_cast<uint16_t*>(epi);
-      for (int c = 0; c < kToks / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * kToks + c * 32, v);
-        tmem_wait_ld();
+      const uint32_t st = smem_u32(epi);
+      for (int hf = 0; hf < kToks / kEpiToks; ++hf) {
+        if (leader) bulk_wait_read0();  // the previous store has read the staging buffer
+        named_barrier(2, 128);
+        for (int c = 0; c < kEpiToks / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * kToks +
+                        hf * kEpiToks + c * 32,
+                    v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
-          st[(c * 32 + i) * kRows + row] = *reinterpret_cast<uint16_t*>(&h);
+          for (int i = 0; i < 32; ++i) {
+            __nv_bfloat16 hv = __float2bfloat16_rn(__uint_as_float(v[i]));
+            sts16(st + ((c * 32 + i) * kRows + row) * 2, *reinterpret_cast<uint16_t*>(&hv));
+          }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
-      fence_async_smem();
-      named_barrier(2, 128);
-      if (leader) {
-        tma_store_2d(&tmY, epi, nt * kRows, mt * kToks);
-        bulk_commit();
+        if (hf == kToks / kEpiToks - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
+        }
+        fence_async_smem();
+        named_barrier(2, 128);
+        if (leader) {
+          tma_store_2d(&tmY, epi, nt * kRows, mt * kToks + hf * kEpiToks);
+          bulk_commit();
+        }
       }
     }
     if (leader) bulk_wait0();
@@ -408,14 +450,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 bool make_map(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+  const CUresult r = fn(map, dtype, 2, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -430,20 +473,30 @@ wq_status launch_tc_gemm(const TcGemmArgs& a, int sms, unsigned* status, cudaStr
   if (!int8 && a.sz_row && a.group % 32 != 0) return WQ_ERR_SHAPE;
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!al16(a.X) || !al16(a.Y) || a.ldx % 8 != 0 || a.ldy % 8 != 0) return WQ_ERR_ALIGN;
-  CUtensorMap mx, my;
+  if (!al16(int8 ? static_cast<const void*>(a.Q8) : static_cast<const void*>(a.P)))
+    return WQ_ERR_ALIGN;
+  CUtensorMap mx, my, mw;
   if (!make_map(&mx, a.X, a.K, a.M, a.ldx * 2, kBK, kToks, true)) return WQ_ERR_CUDA;
-  if (!make_map(&my, a.Y, a.N, a.M, a.ldy * 2, kRows, kToks, false)) return WQ_ERR_CUDA;
+  if (!make_map(&my, a.Y, a.N, a.M, a.ldy * 2, kRows, kEpiToks, false)) return WQ_ERR_CUDA;
+  if (int8) {
+    if (!make_map(&mw, a.Q8, a.K, a.N, a.K, kBK, kRows, false, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+      return WQ_ERR_CUDA;
+  } else if (!make_map(&mw, a.P, a.K / 2, a.N, a.K / 2, kBK / 2, kRows, false,
+                       CU_TENSOR_MAP_DATA_TYPE_UINT8)) {
+    return WQ_ERR_CUDA;
+  }
   auto kern = int8 ? tc_gemm_kernel<true> : tc_gemm_kernel<false>;
+  const size_t smem = int8 ? smem_bytes<true>() : smem_bytes<false>();
   static bool attr[2] = {false, false};
   if (!attr[int8]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+                             static_cast<int>(smem)) != cudaSuccess)
       return WQ_ERR_CUDA;
     attr[int8] = true;
   }
   const int tiles = ((a.N + kRows - 1) / kRows) * ((a.M + kToks - 1) / kToks);
   const int grid = tiles < sms ? tiles : sms;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(mx, my, a.P, a.Q8, a.S, a.Z, a.M, a.N, a.K, a.group,
+  kern<<<grid, kThreads, smem, st>>>(mx, my, mw, a.P, a.Q8, a.S, a.Z, a.M, a.N, a.K, a.group,
                                            a.sz_row, status);
   return cudaGetLastError() == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
