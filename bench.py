@@ -458,7 +458,7 @@ def run_gpu(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                         "peak_source": peak_src, "kernel": "gemv_m1_bulk (M=1)"},
+                         "peak_source": peak_src, "kernel": "gemv_mma_bulk (M=1)"},
             "per_shape": per_shape,
             "secondary": secondary,
             "clocks": dict(clk.summary(), **({"soak_steps_after_timed_region": soak}

@@ -309,6 +309,422 @@ gemv_m1_bulk(const uint16_t* __restrict__ X, const uint8_t* __restrict__ P,
   }
 }
 
+// Small-M W4A16 matmul on the tensor cores' warp-level MMA (m16n8k16, bf16 x bf16 -> fp32),
+// for decode: the CUDA-core form above needs ~2.3 instructions per weight (a byte-permute
+// per code plus the FMAs); here a pair of codes becomes a bf16 pair (128 + q) with one LOP3,
+// and one MMA consumes 256 weights per warp. M <= 8 tokens occupy the MMA's N = 8 columns.
+//
+// Layout of the work: a warp processes one 16-row tile of W against one group (128 k) per
+// step: lane (r = lane/4, c = lane%4) loads bytes [16c, 16c + 16) of the group's 64 bytes for
+// rows r and r + 8 (each load instruction reads 8 rows x 64 contiguous bytes). A 32-bit word
+// holds 8 consecutive codes k0..k7; it unpacks to the pairs (k0,k4), (k1,k5), (k2,k6),
+// (k3,k7). MMA j of the group (j = 0..7) takes pairs from word j/2 of the lane's 4 words; the
+// X operand is permuted identically once per CTA into shared memory ("fragment order"), so
+// the k order inside the MMA is irrelevant to the sum. One packed bf16 subtraction per pair
+// turns (128 + q) into the exact small integer q - Z of its row, so each group's fp32 result
+// is D = sum (q - Z) x with no large offset to cancel, and S' is applied once per group:
+// acc += S' D.
+// The CTA (8 warps) owns a 16-row tile, its warps split the groups, and the partial tiles
+// are summed through shared memory in a fixed order.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// (128 + q) bf16 pairs of a word's codes: out[i] = (k_i, k_{i+4}) for i = 0..3.
+__device__ __forceinline__ void unpack_bf16_pairs(uint32_t w, uint32_t (&out)[4]) {
+  out[0] = (w & 0x000F000Fu) | 0x43004300u;
+  out[1] = ((w >> 4) & 0x000F000Fu) | 0x43004300u;
+  out[2] = ((w >> 8) & 0x000F000Fu) | 0x43004300u;
+  out[3] = ((w >> 12) & 0x000F000Fu) | 0x43004300u;
+}
+
+template <int M>
+__global__ void __launch_bounds__(256)
+gemv_mma(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restrict__ P,
+         const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int N, int K,
+         int group, int sz_row, uint16_t* __restrict__ Y, int64_t ldy) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int G = K / 128;
+  uint32_t* xf = reinterpret_cast<uint32_t*>(smem);                      // [G][4M][16]
+  float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(G) * 4 * M * 64);  // [8][16][8]
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- X -> fragment order (once per CTA) and per-group token sums
+  for (int e = threadIdx.x; e < G * 4 * M; e += blockDim.x) {
+    const int g = e / (4 * M);
+    const int L = e - g * 4 * M;  // fragment lane: token n = L/4, quarter c = L%4
+    const int n = L >> 2, c = L & 3;
+    const uint16_t* xs = X + n * ldx + g * 128 + 32 * c;
+    uint32_t xw[16];  // x[32c + 2i], x[32c + 2i + 1] pairs
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 u = ld_nc_u4(xs + 8 * v);
+      xw[4 * v] = u.x; xw[4 * v + 1] = u.y; xw[4 * v + 2] = u.z; xw[4 * v + 3] = u.w;
+    }
+    uint32_t* dst = xf + (static_cast<size_t>(g) * 4 * M + L) * 16;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      // word w = j/2 covers x[32c + 8w .. +7] = xw[4w .. 4w+3]; pairs (k, k+4) with
+      // k = 2(j%2) (b0) and 2(j%2) + 1 (b1)
+      const int w = j >> 1, o = (j & 1) * 2;
+      const uint32_t lo = xw[4 * w + (o >> 1)];      // (x[8w+o], x[8w+o+1])
+      const uint32_t hi = xw[4 * w + 2 + (o >> 1)];  // (x[8w+o+4], x[8w+o+5])
+      dst[2 * j] = __byte_perm(lo, hi, 0x5410);      // (x[8w+o], x[8w+o+4])
+      dst[2 * j + 1] = __byte_perm(lo, hi, 0x7632);  // (x[8w+o+1], x[8w+o+5])
+    }
+  }
+  __syncthreads();
+
+  const int r = lane >> 2, c = lane & 3;
+  const int t0 = 2 * c, t1 = 2 * c + 1;  // tokens (columns) of this lane's accumulators
+  const int g_lo = (warp * G) / 8, g_hi = ((warp + 1) * G) / 8;
+  const int ntiles = (N + 15) / 16;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int n0 = tile * 16 + r, n1 = n0 + 8;
+    const bool v0 = n0 < N, v1 = n1 < N;
+    const uint8_t* p0 = P + static_cast<int64_t>(n0) * (K / 2) + 16 * c;
+    const uint8_t* p1 = P + static_cast<int64_t>(n1) * (K / 2) + 16 * c;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint4 wa = make_uint4(0, 0, 0, 0), wb = wa;
+    if (g_lo < g_hi) {
+      if (v0) wa = ld_stream_u4(p0 + g_lo * 64);
+      if (v1) wb = ld_stream_u4(p1 + g_lo * 64);
+    }
+    for (int g = g_lo; g < g_hi; ++g) {
+      const uint4 ca = wa, cb = wb;
+      if (g + 1 < g_hi) {  // next group's codes in flight while this one computes
+        if (v0) wa = ld_stream_u4(p0 + (g + 1) * 64);
+        if (v1) wb = ld_stream_u4(p1 + (g + 1) * 64);
+      }
+      const int64_t gi0 = static_cast<int64_t>(n0) * sz_row + (sz_row ? (g * 128) / group : 0);
+      const int64_t gi1 = static_cast<int64_t>(n1) * sz_row + (sz_row ? (g * 128) / group : 0);
+      const float s0 = v0 ? f16_bits_to_f32(ld_nc_u16(S + gi0)) : 0.0f;
+      const float z0 = v0 ? f16_bits_to_f32(ld_nc_u16(Zp + gi0)) : 0.0f;
+      const float s1 = v1 ? f16_bits_to_f32(ld_nc_u16(S + gi1)) : 0.0f;
+      const float z1 = v1 ? f16_bits_to_f32(ld_nc_u16(Zp + gi1)) : 0.0f;
+      const __nv_bfloat162 zz0 = __floats2bfloat162_rn(128.0f + z0, 128.0f + z0);
+      const __nv_bfloat162 zz1 = __floats2bfloat162_rn(128.0f + z1, 128.0f + z1);
+      uint4 xb[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                     make_uint4(0, 0, 0, 0)};
+      if (lane < 4 * M) {
+        const uint4* src = reinterpret_cast<const uint4*>(xf + (static_cast<size_t>(g) * 4 * M + lane) * 16);
+        xb[0] = src[0]; xb[1] = src[1]; xb[2] = src[2]; xb[3] = src[3];
+      }
+      const uint32_t bw[16] = {xb[0].x, xb[0].y, xb[0].z, xb[0].w, xb[1].x, xb[1].y, xb[1].z, xb[1].w,
+                               xb[2].x, xb[2].y, xb[2].z, xb[2].w, xb[3].x, xb[3].y, xb[3].z, xb[3].w};
+      const uint32_t wr0[4] = {ca.x, ca.y, ca.z, ca.w};
+      const uint32_t wr1[4] = {cb.x, cb.y, cb.z, cb.w};
+      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t pa[4], pb[4];
+        unpack_bf16_pairs(wr0[w], pa);
+        unpack_bf16_pairs(wr1[w], pb);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // (128 + q) - (128 + Z) = q - Z, exact in bf16
+          __nv_bfloat162 ta = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&pa[i]), zz0);
+          __nv_bfloat162 tb = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&pb[i]), zz1);
+          pa[i] = *reinterpret_cast<uint32_t*>(&ta);
+          pb[i] = *reinterpret_cast<uint32_t*>(&tb);
+        }
+        const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
+        const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
+        mma_bf16_16816(d, a0, bw[4 * w], bw[4 * w + 1]);
+        mma_bf16_16816(d, a1, bw[4 * w + 2], bw[4 * w + 3]);
+      }
+      acc[0] = fmaf(s0, d[0], acc[0]);
+      acc[1] = fmaf(s0, d[1], acc[1]);
+      acc[2] = fmaf(s1, d[2], acc[2]);
+      acc[3] = fmaf(s1, d[3], acc[3]);
+    }
+    // partial tile of this warp -> shared; sum over the 8 warps in a fixed order
+    float* rw = red + warp * 128;
+    rw[r * 8 + t0] = acc[0];
+    rw[r * 8 + t1] = acc[1];
+    rw[(r + 8) * 8 + t0] = acc[2];
+    rw[(r + 8) * 8 + t1] = acc[3];
+    __syncthreads();
+    if (threadIdx.x < 16 * M) {
+      const int row = threadIdx.x / M, tok = threadIdx.x - (threadIdx.x / M) * M;
+      float t = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) t += red[w * 128 + row * 8 + tok];
+      const int n = tile * 16 + row;
+      if (n < N) {
+        __nv_bfloat16 hv = __float2bfloat16_rn(t);
+        Y[tok * ldy + n] = *reinterpret_cast<uint16_t*>(&hv);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Small-M W4A16 matmul: warp-level MMA consumers fed by bulk asynchronous copies.
+// One producer lane streams 16-row tiles into a shared-memory ring: each row's K/2 packed
+// bytes land at a row stride of 64 mod 128 bytes (so the MMA warps' 16-byte reads are
+// bank-conflict free) and the tile's S' and Z (16 x G each, contiguous in HBM) follow.
+// Sixteen MMA warps split the tile's groups. Codes are decoded with the bf16 magic
+// 1 + q/16 (nibble in the top mantissa bits: one shift and one LOP3 per pair of codes), so
+// one group's MMA result is D = sum x (1 + q/16) and, with sum x of the group,
+//   sum x (q - Z) = 16 D - (16 + Z) sum x,      acc += S' (16 D - (16 + Z) sum x).
+// The offset is small (16 against q - Z), so the fp32 cancellation costs only a few bits.
+// The X fragments (see gemv_mma) and the per-group token sums are built once per CTA.
+// Each group's 8 MMAs run as two independent accumulator chains.
+// (a & b) | c in one 3-input logic op (both constants arrive in registers, so no second op).
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// (1 + q/16) bf16 pairs of a word's codes: out[i] = (k_i, k_{i+4}) for i = 0..3.
+// mask = 0x00780078, magic = 0x3F803F80 (passed in registers by the caller).
+__device__ __forceinline__ void unpack_bf16_hi(uint32_t w, uint32_t mask, uint32_t magic,
+                                               uint32_t (&out)[4]) {
+  out[0] = and_or(w << 3, mask, magic);
+  out[1] = and_or(w >> 1, mask, magic);
+  out[2] = and_or(w >> 5, mask, magic);
+  out[3] = and_or(w >> 9, mask, magic);
+}
+
+// Shared-memory layout of gemv_mma_bulk (host and device agree through this).
+struct MmaBulkLayout {
+  uint32_t xf_bytes, sx_bytes, stage_bytes, wbytes, szbytes, ring_off, bar_off, red_off, total;
+  __host__ __device__ MmaBulkLayout(int M, int K, int wstride, int stages, int NW, int RT) {
+    const uint32_t G = K / 128;
+    xf_bytes = G * 4 * M * 64;
+    sx_bytes = G * 8 * 4;
+    wbytes = 16u * RT * wstride;
+    szbytes = 16u * RT * G * 2;
+    stage_bytes = wbytes + 2 * szbytes;
+    ring_off = xf_bytes + sx_bytes;
+    bar_off = ring_off + stages * stage_bytes;
+    red_off = bar_off + (2 * stages + 2) * 8;
+    total = red_off + 2u * NW * RT * 16 * (M < 2 ? 2 : M) * 4;
+  }
+};
+
+// Small-M W4A16 matmul: warp-level MMA consumers fed by bulk asynchronous copies.
+// One producer lane streams tiles of 16*RT rows into a shared-memory ring: each row's K/2
+// packed bytes land at a row stride of 64 mod 128 bytes (so the MMA warps' 16-byte reads
+// are bank-conflict free), followed by the tile's S' and Z (contiguous in HBM). NW MMA
+// warps split the groups of K; per group a warp decodes and multiplies all RT 16-row
+// sub-tiles, so the X fragments are read once per group and the RT accumulator chains are
+// independent. Codes are decoded with the bf16 magic 1 + q/16 (nibble in the top mantissa
+// bits: one shift and one 3-input LOP3 per pair of codes), so a group's MMA result is
+// D = sum x (1 + q/16) and, with the group's sum of x,
+//   sum x (q - Z) = 16 D - (16 + Z) sum x,      acc += S' (16 D - (16 + Z) sum x).
+// The offset is small (16 against q - Z), so the fp32 cancellation costs only a few bits.
+// Partial tiles are summed over the warps in shared memory behind a bounded mbarrier.
+template <int M, int NW, int RT>
+__global__ void __launch_bounds__(32 * (NW + 1), 1)
+gemv_mma_bulk(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restrict__ P,
+              const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int N, int K,
+              int wstride, int stages, uint32_t prefetch_bytes, uint16_t* __restrict__ Y,
+              int64_t ldy, unsigned* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int MR = M < 2 ? 2 : M;  // token slots kept in the reduction buffer
+  constexpr int TR = 16 * RT;        // rows per tile
+  const MmaBulkLayout L(M, K, wstride, stages, NW, RT);
+  const int G = K / 128;
+  uint32_t* xf = reinterpret_cast<uint32_t*>(smem);                  // [G][4M][16]
+  float* sxs = reinterpret_cast<float*>(smem + L.xf_bytes);           // [G][8]
+  uint8_t* ring = smem + L.ring_off;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint64_t* empty = full + stages;
+  uint64_t* redbar = empty + stages;  // [2]
+  float* red = reinterpret_cast<float*>(smem + L.red_off);  // [2][NW][TR][MR]
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ntiles = N / TR;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], NW);
+    }
+    mbar_init(&redbar[0], NW);
+    mbar_init(&redbar[1], NW);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Let the next kernel on the stream launch now; warm L2 with this CTA's weight tiles
+  // (a hint, safe before the dependency wait), then wait for the previous kernel.
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  const uint32_t tile_w = static_cast<uint32_t>(TR) * (K / 2);
+  if (warp == NW && lane == 0) {
+    uint32_t budget = prefetch_bytes;
+    for (int tile = blockIdx.x; tile < ntiles && budget >= tile_w; tile += gridDim.x) {
+      prefetch_l2_bulk(P + static_cast<int64_t>(tile) * tile_w, tile_w);
+      budget -= tile_w;
+    }
+  }
+  pdl_wait();
+
+  if (warp == NW) {  // producer
+    if (lane == 0) {
+      int i = 0;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+        const int st = i % stages;
+        const uint32_t use = i / stages;
+        if (use > 0 && !mbar_wait_bounded(&empty[st], (use - 1) & 1u, kWaitLimitNs)) {
+          set_status(status, kStTimeout);
+          break;
+        }
+        uint8_t* dst = ring + static_cast<size_t>(st) * L.stage_bytes;
+        mbar_arrive_expect_tx(&full[st], tile_w + 2 * L.szbytes);
+        const uint8_t* src = P + static_cast<int64_t>(tile) * tile_w;
+        for (int r = 0; r < TR; ++r)
+          bulk_g2s(dst + r * wstride, src + static_cast<int64_t>(r) * (K / 2), K / 2, &full[st]);
+        bulk_g2s(dst + L.wbytes, S + static_cast<int64_t>(tile) * TR * G, L.szbytes, &full[st]);
+        bulk_g2s(dst + L.wbytes + L.szbytes, Zp + static_cast<int64_t>(tile) * TR * G,
+                 L.szbytes, &full[st]);
+      }
+      for (int st = 0; st < stages && st < i; ++st) {
+        const uint32_t last = (i - 1 - st) / stages;
+        if (!mbar_wait_bounded(&full[st], last & 1u, kWaitLimitNs)) set_status(status, kStTimeout);
+      }
+    }
+    return;
+  }
+
+  // X -> fragment order and per-group token sums; overlaps with the producer's first copies
+  for (int e = threadIdx.x; e < G * 4 * M; e += 32 * NW) {
+    const int g = e / (4 * M);
+    const int Lf = e - g * 4 * M;
+    const int n = Lf >> 2, c = Lf & 3;
+    const uint16_t* xs = X + n * ldx + g * 128 + 32 * c;
+    uint32_t xw[16];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 u = ld_nc_u4(xs + 8 * v);
+      xw[4 * v] = u.x; xw[4 * v + 1] = u.y; xw[4 * v + 2] = u.z; xw[4 * v + 3] = u.w;
+    }
+    uint32_t* dst = xf + (static_cast<size_t>(g) * 4 * M + Lf) * 16;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int w = j >> 1, o = (j & 1) * 2;
+      const uint32_t lo = xw[4 * w + (o >> 1)];
+      const uint32_t hi = xw[4 * w + 2 + (o >> 1)];
+      dst[2 * j] = __byte_perm(lo, hi, 0x5410);
+      dst[2 * j + 1] = __byte_perm(lo, hi, 0x7632);
+    }
+  }
+  for (int e = threadIdx.x; e < G * 8; e += 32 * NW) {
+    const int g = e >> 3, n = e & 7;
+    float t = 0.0f;
+    if (n < M) {
+      const uint16_t* xs = X + n * ldx + g * 128;
+      uint4 u[16];
+#pragma unroll
+      for (int v = 0; v < 16; ++v) u[v] = ld_nc_u4(xs + 8 * v);
+#pragma unroll
+      for (int v = 0; v < 16; ++v)
+        t += ((bf16_lo(u[v].x) + bf16_hi(u[v].x)) + (bf16_lo(u[v].y) + bf16_hi(u[v].y))) +
+             ((bf16_lo(u[v].z) + bf16_hi(u[v].z)) + (bf16_lo(u[v].w) + bf16_hi(u[v].w)));
+    }
+    sxs[e] = t;
+  }
+  named_barrier(1, 32 * NW);
+
+  const int r = lane >> 2, c = lane & 3;
+  const int t0 = 2 * c, t1 = 2 * c + 1;
+  const int g_lo = (warp * G) / NW, g_hi = ((warp + 1) * G) / NW;
+  // lanes whose token column is >= M read a duplicate fragment: their columns are never
+  // stored, and the loads stay uniform (no divergent branch)
+  const uint32_t xf_lane = smem_u32(xf) + (lane % (4 * M)) * 64;
+  const uint32_t ring_s = smem_u32(ring);
+  const float* sx0p = sxs + t0;
+  const float* sx1p = sxs + t1;
+  uint32_t kMask = 0x00780078u, kMagic = 0x3F803F80u;  // register operands of the LOP3
+  asm volatile("" : "+r"(kMask), "+r"(kMagic));
+  int i = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+    const int st = i % stages;
+    if (!mbar_wait_bounded(&full[st], (i / stages) & 1u, kWaitLimitNs)) {
+      set_status(status, kStTimeout);
+      return;
+    }
+    const uint32_t wb = ring_s + st * L.stage_bytes;
+    const uint32_t sb = wb + L.wbytes, zb = sb + L.szbytes;
+    float acc[RT][4];
+#pragma unroll
+    for (int t = 0; t < RT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+    for (int g = g_lo; g < g_hi; ++g) {
+      const uint32_t xs = xf_lane + g * (4 * M * 64);
+      const uint4 xb0 = lds128(xs), xb1 = lds128(xs + 16), xb2 = lds128(xs + 32),
+                  xb3 = lds128(xs + 48);
+      const uint32_t bw[16] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w,
+                               xb2.x, xb2.y, xb2.z, xb2.w, xb3.x, xb3.y, xb3.z, xb3.w};
+      const float sx0 = sx0p[g * 8], sx1 = sx1p[g * 8];
+#pragma unroll
+      for (int t = 0; t < RT; ++t) {
+        const int ra = 16 * t + r, rb = ra + 8;
+        const uint4 ca = lds128(wb + ra * wstride + g * 64 + 16 * c);
+        const uint4 cb = lds128(wb + rb * wstride + g * 64 + 16 * c);
+        const uint32_t wr0[4] = {ca.x, ca.y, ca.z, ca.w};
+        const uint32_t wr1[4] = {cb.x, cb.y, cb.z, cb.w};
+        float de[4] = {0.0f, 0.0f, 0.0f, 0.0f}, dodd[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          uint32_t pa[4], pb[4];
+          unpack_bf16_hi(wr0[w], kMask, kMagic, pa);
+          unpack_bf16_hi(wr1[w], kMask, kMagic, pb);
+          const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
+          const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
+          mma_bf16_16816(de, a0, bw[4 * w], bw[4 * w + 1]);
+          mma_bf16_16816(dodd, a1, bw[4 * w + 2], bw[4 * w + 3]);
+        }
+        const float s0 = f16_bits_to_f32(lds16(sb + (ra * G + g) * 2));
+        const float z0 = f16_bits_to_f32(lds16(zb + (ra * G + g) * 2));
+        const float s1 = f16_bits_to_f32(lds16(sb + (rb * G + g) * 2));
+        const float z1 = f16_bits_to_f32(lds16(zb + (rb * G + g) * 2));
+        acc[t][0] = fmaf(s0, fmaf(16.0f, de[0] + dodd[0], -(16.0f + z0) * sx0), acc[t][0]);
+        acc[t][1] = fmaf(s0, fmaf(16.0f, de[1] + dodd[1], -(16.0f + z0) * sx1), acc[t][1]);
+        acc[t][2] = fmaf(s1, fmaf(16.0f, de[2] + dodd[2], -(16.0f + z1) * sx0), acc[t][2]);
+        acc[t][3] = fmaf(s1, fmaf(16.0f, de[3] + dodd[3], -(16.0f + z1) * sx1), acc[t][3]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+    const int par = i & 1;
+    float* rw = red + (par * NW + warp) * TR * MR;
+#pragma unroll
+    for (int t = 0; t < RT; ++t) {
+      const int ra = 16 * t + r, rb = ra + 8;
+      if (t0 < M) {
+        rw[ra * MR + t0] = acc[t][0];
+        rw[rb * MR + t0] = acc[t][2];
+      }
+      if (t1 < M) {
+        rw[ra * MR + t1] = acc[t][1];
+        rw[rb * MR + t1] = acc[t][3];
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&redbar[par]);
+    if (!mbar_wait_bounded(&redbar[par], (i >> 1) & 1u, kWaitLimitNs)) {
+      set_status(status, kStTimeout);
+      return;
+    }
+    for (int e = threadIdx.x; e < TR * M; e += 32 * NW) {
+      const int row = e / M, tok = e - (e / M) * M;
+      const float* rp = red + par * NW * TR * MR + row * MR + tok;
+      float t = 0.0f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) t += rp[w * TR * MR];
+      __nv_bfloat16 hv = __float2bfloat16_rn(t);
+      Y[tok * ldy + tile * TR + row] = *reinterpret_cast<uint16_t*>(&hv);
+    }
+  }
+}
+
 template <int M>
 __global__ void __launch_bounds__(256)
 gemv_rows(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restrict__ P,
@@ -484,6 +900,95 @@ cudaError_t launch_m1_bulk(const GemvArgs& a, int sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+size_t mma_smem(int M, int K) {
+  const size_t G = K / 128;
+  return G * 4 * M * 64 + 8 * 128 * 4;
+}
+
+template <int M>
+cudaError_t launch_mma(const GemvArgs& a, int sms, cudaStream_t st) {
+  const size_t smem = mma_smem(M, a.K);
+  static int occ_cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& occ = occ_cache[dev & 63];
+  if (occ == 0) {
+    cudaFuncSetAttribute(gemv_mma<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    occ = -1;
+  }
+  int o = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_mma<M>, 256, smem) != cudaSuccess ||
+      o < 1)
+    o = 1;
+  const int ntiles = (a.N + 15) / 16;
+  int grid = sms * o;
+  if (grid > ntiles) grid = ntiles;
+  gemv_mma<M><<<grid, 256, smem, st>>>(a.X, a.ldx, a.P, a.S, a.Z, a.N, a.K, a.group, a.sz_row,
+                                       a.Y, a.ldy);
+  return cudaGetLastError();
+}
+
+template <int M, int NW, int RT>
+cudaError_t launch_mma_bulk(const GemvArgs& a, int sms, cudaStream_t st) {
+  const int half = a.K / 2;
+  const int wstride = half + ((64 - half % 128) + 128) % 128;  // = 64 (mod 128)
+  constexpr size_t kBudget = 220 * 1024;  // one CTA per SM
+  int stages = 8;
+  while (stages >= 2 && MmaBulkLayout(M, a.K, wstride, stages, NW, RT).total > kBudget) --stages;
+  if (stages < 2) return cudaErrorInvalidValue;
+  const size_t smem = MmaBulkLayout(M, a.K, wstride, stages, NW, RT).total;
+  auto kern = gemv_mma_bulk<M, NW, RT>;
+  static bool attr[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr[dev & 63]) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kBudget));
+    attr[dev & 63] = true;
+  }
+  const int ntiles = a.N / (16 * RT);
+  const int grid = ntiles < sms ? ntiles : sms;
+  // L2 warm-up per CTA: at most 48 MB for the whole grid
+  const uint32_t prefetch = static_cast<uint32_t>((48ull << 20) / grid);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(32 * (NW + 1));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a.X, a.ldx, a.P, a.S, a.Z, a.N, a.K, wstride, stages,
+                            prefetch, a.Y, a.ldy, a.status);
+}
+
+// MMA warps per CTA of the bulk-fed decode kernel. Tiles are 32 rows when two stages of
+// them fit in shared memory (more work per fragment load and per sync), else 16 rows.
+constexpr int kDecodeWarps = 8;
+
+template <int M>
+cudaError_t launch_mma_bulk_any(const GemvArgs& a, int sms, cudaStream_t st) {
+  if (a.N % 32 == 0) {
+    const cudaError_t e = launch_mma_bulk<M, kDecodeWarps, 2>(a, sms, st);
+    if (e != cudaErrorInvalidValue) return e;
+  }
+  return launch_mma_bulk<M, kDecodeWarps, 1>(a, sms, st);
+}
+
+bool mma_bulk_ok(const GemvArgs& a) {
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  return a.K % 128 == 0 && a.sz_row > 0 && a.group == 128 && a.N % 16 == 0 &&
+         (a.ldx % 8) == 0 && al16(a.X) && al16(a.P) && al16(a.S) && al16(a.Z);
+}
+
+bool mma_ok(const GemvArgs& a) {
+  return a.K % 128 == 0 && (a.sz_row == 0 || a.group % 128 == 0) &&
+         mma_smem(a.M, a.K) <= 96 * 1024 && (a.ldx % 8) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.X) & 15u) == 0;
+}
+
 bool bulk_ok(const GemvArgs& a) {
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   return a.M == 1 && a.N % 8 == 0 && a.sz_row > 0 && a.K <= 16 * 1024 && al16(a.P) &&
@@ -509,6 +1014,34 @@ cudaError_t launch_gemv_w8a16(const Gemv8Args& a, cudaStream_t st) {
 int gemv_max_k() { return 32 * kSlice; }
 
 cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st) {
+  if (mma_bulk_ok(a)) {
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (a.M) {
+      case 1: e = launch_mma_bulk_any<1>(a, sms, st); break;
+      case 2: e = launch_mma_bulk_any<2>(a, sms, st); break;
+      case 3: e = launch_mma_bulk_any<3>(a, sms, st); break;
+      case 4: e = launch_mma_bulk_any<4>(a, sms, st); break;
+      case 5: e = launch_mma_bulk_any<5>(a, sms, st); break;
+      case 6: e = launch_mma_bulk_any<6>(a, sms, st); break;
+      case 7: e = launch_mma_bulk_any<7>(a, sms, st); break;
+      case 8: e = launch_mma_bulk_any<8>(a, sms, st); break;
+      default: break;
+    }
+    if (e != cudaErrorInvalidValue) return e;
+  }
+  if (mma_ok(a)) {
+    switch (a.M) {
+      case 1: return launch_mma<1>(a, sms, st);
+      case 2: return launch_mma<2>(a, sms, st);
+      case 3: return launch_mma<3>(a, sms, st);
+      case 4: return launch_mma<4>(a, sms, st);
+      case 5: return launch_mma<5>(a, sms, st);
+      case 6: return launch_mma<6>(a, sms, st);
+      case 7: return launch_mma<7>(a, sms, st);
+      case 8: return launch_mma<8>(a, sms, st);
+      default: break;
+    }
+  }
   switch (a.M) {
     case 1:
       if (bulk_ok(a)) {

@@ -81,6 +81,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// As mbar_wait_bounded, for short latency-critical handoffs: polls without asking the
+// hardware to suspend the warp (whose wake-up is coarser than a spin), reading the timer
+// only every 64 polls.
+__device__ __forceinline__ bool mbar_wait_spin_bounded(uint64_t* bar, uint32_t parity,
+                                                       uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // Shared-memory 16-byte load / store by shared-window address.
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -112,6 +125,19 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Programmatic dependent launch: let the next kernel on the stream start launching, and
+// wait until every prerequisite grid has completed with its memory visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Hint: bring `bytes` (multiple of 16, 16-byte aligned) of global memory into L2. Only a
+// hint, so it is safe before pdl_wait(): L2 is coherent with any later writes.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // Barrier over `threads` threads (a multiple of 32) using hardware barrier `id` (1..15).
