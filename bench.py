@@ -476,6 +476,57 @@ def run_gpu(args):
     return 0
 
 
+CASES = ("quantize_70b", "gemv_m1_7b", "gemv_m4_7b", "gemv_m16_7b", "prefill", "prefill_w8")
+
+
+def run_case(name, reps):
+    """Launch one kernel family `reps` times on one named workload, untimed, for a profiler
+    to capture (e.g. ncu -k <kernel> -s <skip> -c <count> python bench.py --case NAME)."""
+    import torch
+
+    import w4a16_dequant_matmul_b200 as wq
+
+    wq.build_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def bf16(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    if name == "quantize_70b":
+        N, K = wq_inputs.SHAPES_70B[0]
+        Wt = (torch.randn(N, K, device=dev) * 0.015).to(torch.bfloat16)
+        p = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        s = torch.empty((N, K // 128), dtype=torch.float16, device=dev)
+        z = torch.empty_like(s)
+        for _ in range(reps):
+            wq.wq_quantize_rtn_g128(Wt, packed=p, S=s, Z=z)
+    elif name.startswith("gemv_m"):
+        M = int(name[len("gemv_m"):].split("_")[0])
+        work = []
+        for (N, K) in SHAPES:
+            packed, S, Z = wq.wq_quantize_rtn_g128(bf16(wq_inputs.weight_bf16(N, K, 0.02)))
+            work.append((bf16(wq_inputs.act_bf16(M, K)), packed, S, Z))
+        for _ in range(reps):
+            for (X, packed, S, Z) in work:
+                wq.wq_w4a16_gemm(X, packed, S, Z, 128)
+    else:
+        P = wq_inputs.PREFILL
+        Wt = (torch.randn(P["N"], P["K"], device=dev) * 0.02).to(torch.bfloat16)
+        Xp = torch.randn(P["M"], P["K"], device=dev).to(torch.bfloat16)
+        if name == "prefill":
+            pk, s, z = wq.wq_quantize_rtn_g128(Wt)
+            for _ in range(reps):
+                wq.wq_w4a16_gemm(Xp, pk, s, z, 128)
+        else:
+            q, s, _ = wq.wq_quantize_rtn_g128(Wt, 8, P["K"], False)
+            for _ in range(reps):
+                wq.wq_w8a16_gemm(Xp, q, s)
+    torch.cuda.synchronize()
+    st = wq.wq_get_status()
+    print(f"case {name}: {reps} reps, status {st}")
+    return 0 if st == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -485,7 +536,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-soak", action="store_true",
                     help="no clock soak after a short timed region (for profiler runs)")
+    ap.add_argument("--case", choices=CASES,
+                    help="only launch this workload's kernel --case-reps times (profiling)")
+    ap.add_argument("--case-reps", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        return run_case(args.case, args.case_reps)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -92,6 +92,36 @@ def test_adversarial_groups(dtype):
         _check_int4(W.astype(np.float64), gu.f32(W), g)
 
 
+def _tie_lattice_bits():
+    """bf16 groups rich in exact and near half-integer quotients w/S'.
+
+    Each 128-group is built around S0 = m 2^e (m odd, up to 8 bits) and Z0 in 0..15: its
+    ends -Z0 S0 and (15 - Z0) S0, every (k + 1/2) S0 in between, and uniform fill. After the
+    cast to bf16 many values are exact ties of the group's S' and the rest lie within a few
+    ulps of one; a second copy moves half the weights one bf16 ulp up or down."""
+    rng = np.random.default_rng(99)
+    groups = []
+    for m in (1, 3, 5, 7, 9, 11, 13, 15, 17, 25, 31, 63, 127, 255):
+        for e in (-22, -12, -5, 0, 4):
+            for z in range(16):
+                s0 = m * 2.0 ** e
+                vals = [-z * s0, (15 - z) * s0] + [(k + 0.5) * s0 for k in range(-z, 15 - z)]
+                g = np.resize(np.array(vals), 128)
+                g[len(vals):] = rng.uniform(-z * s0, (15 - z) * s0, 128 - len(vals))
+                groups.append(g)
+    bits = wq_inputs.to_bf16_bits(np.array(groups).reshape(-1, 256)).astype(np.int32)
+    move = (rng.random(bits.shape) < 0.5) & ((bits & 0x7FFF) != 0)
+    step = np.where(rng.random(bits.shape) < 0.5, 1, -1)
+    return np.concatenate([bits, np.where(move, bits + step, bits)]).astype(np.uint16)
+
+
+def test_tie_lattice_bf16():
+    """Round-half-even decisions on exact ties and their bf16 neighbours, every Z parity,
+    clipped and unclipped groups."""
+    Wb = _tie_lattice_bits()
+    _check_int4(wq_inputs.bf16_bits_to_f64(Wb), gu.bf16_from_bits(Wb), 128)
+
+
 def test_strided_rows():
     """ldw > K: W is a column slice of a wider matrix."""
     big = wq_inputs.to_f32(wq_inputs.normal_f64((20, 640), 0.02, 4))

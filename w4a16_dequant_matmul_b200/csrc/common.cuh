@@ -80,10 +80,13 @@ __device__ __forceinline__ double exact_diff(float hi, float lo, float div, floa
 }
 
 // binary16 bit pattern of round-half-even((hi + lo) / div), where hi >= 0 is finite and lo
-// is the exact rounding error of hi (hi + lo is the exact value). 0x7C00 means overflow.
-static __device__ __noinline__ unsigned rne_f16_of_quotient(float hi, float lo, float div) {
-  // Candidate: within one binary16 step of the answer (float32 error << binary16 step).
-  unsigned b = __half_as_ushort(__float2half_rn(__fdiv_rn(hi, div)));
+// is the exact rounding error of hi (hi + lo is the exact value); rdiv = 1/div rounded to
+// float. 0x7C00 means overflow.
+static __device__ __noinline__ unsigned rne_f16_of_quotient(float hi, float lo, float div,
+                                                            float rdiv) {
+  // Candidate: hi * rdiv is within 2^-23 relative of the quotient, so its binary16
+  // rounding is within one binary16 step of the answer; the two midpoint tests fix it.
+  unsigned b = __half_as_ushort(__float2half_rn(__fmul_rn(hi, rdiv)));
   if (b < 0x7C00u) {
     float m = 0.5f * (f16_grid_value(b) + f16_grid_value(b + 1));
     double d = exact_diff(hi, lo, div, m);
@@ -130,7 +133,7 @@ __device__ __forceinline__ AsymScale asym_scale_zero(float mn, float mx) {
   float hi = a + b;  // exact split of a + b into hi + lo (Fast2Sum, larger operand first)
   float lo = (a >= b) ? (b - (hi - a)) : (a - (hi - b));
   r.bad = !isfinite(hi);
-  unsigned sb = r.bad ? 0x3C00u : rne_f16_of_quotient(hi, lo, 15.0f);
+  unsigned sb = r.bad ? 0x3C00u : rne_f16_of_quotient(hi, lo, 15.0f, 1.0f / 15.0f);
   if (sb >= 0x7C00u) {
     r.bad = true;
     sb = 0x3C00u;
@@ -148,7 +151,7 @@ __device__ __forceinline__ AsymScale asym_scale_zero(float mn, float mx) {
 __device__ __forceinline__ AsymScale sym_scale(float amax, float qmax) {
   AsymScale r;
   r.bad = !isfinite(amax);
-  unsigned sb = r.bad ? 0x3C00u : rne_f16_of_quotient(amax, 0.0f, qmax);
+  unsigned sb = r.bad ? 0x3C00u : rne_f16_of_quotient(amax, 0.0f, qmax, 1.0f / qmax);
   if (sb >= 0x7C00u) {
     r.bad = true;
     sb = 0x3C00u;
