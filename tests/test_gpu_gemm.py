@@ -105,6 +105,46 @@ def test_full_size_decode_sampled(N, K):
     assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref) <= GATE
 
 
+# N a multiple of 16: the streaming decode kernel (16-row tiles, chunks of 4 groups)
+STREAM_SHAPES = [(16, 128), (48, 384), (160, 1152), (32, 11008), (256, 4096)]
+
+
+@pytest.mark.parametrize("N,K", STREAM_SHAPES)
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+def test_stream_tiles_and_chunks(N, K, M):
+    """One tile, ragged last chunks (G = 3, 9, 86 groups), every M of the kernel, X with a
+    row stride above K; bitwise repeatable."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N * 7 + K)
+    Xwide = gu.bf16_from_bits(wq_inputs.act_bf16(M, K + 128, seed=M + 40))
+    X = Xwide[:, 128:]
+    packed, S, Z, codes, So, Zo = _quantize_both(Wb, 128)
+    Y = wq.wq_w4a16_gemm(X, packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    Yref = oracle.w4a16_matmul(gu.bf16_to_f64(X), codes, So, Zo, 128, "exact")
+    y = gu.bf16_to_f64(Y)
+    assert oracle.gemm_gate(y, Yref) <= GATE
+    assert oracle.rel_frobenius(Yref, y) < 4e-3
+    assert torch.equal(Y, wq.wq_w4a16_gemm(X, packed, S, Z, 128))
+
+
+@pytest.mark.parametrize("N,K,M", [(16576, 4096, 1), (11888, 1024, 4), (14208, 256, 2)])
+def test_stream_many_tiles_sampled(N, K, M):
+    """CTAs that own more tiles than there are S'/Z slots and more chunks than ring stages
+    (16576 x 4096: 7 tiles, 56 chunks per CTA on 148 SMs), and a last CTA with fewer tiles;
+    the oracle checks sampled rows, including the first and last."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N)
+    Xb = wq_inputs.act_bf16(M, K, seed=N + 1)
+    packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb))
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    rows = np.sort(np.random.default_rng(N).choice(N, 96, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    codes, So, Zo = oracle.quantize_rtn_asym(wq_inputs.bf16_bits_to_f64(Wb[rows]), 128)
+    np.testing.assert_array_equal(gu.to_np(packed)[rows], oracle.pack_int4(codes))
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "exact")
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref) <= GATE
+
+
 @pytest.mark.parametrize("M", [1, 3, 8])
 def test_w8a16_small_m(M):
     N, K = 130, 2048

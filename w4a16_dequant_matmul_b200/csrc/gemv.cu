@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "mma_frag.cuh"
 
 namespace wq {
 namespace {
@@ -326,15 +327,6 @@ gemv_m1_bulk(const uint16_t* __restrict__ X, const uint8_t* __restrict__ P,
 // acc += S' D.
 // The CTA (8 warps) owns a 16-row tile, its warps split the groups, and the partial tiles
 // are summed through shared memory in a fixed order.
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
-                                               uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // (128 + q) bf16 pairs of a word's codes: out[i] = (k_i, k_{i+4}) for i = 0..3.
 __device__ __forceinline__ void unpack_bf16_pairs(uint32_t w, uint32_t (&out)[4]) {
   out[0] = (w & 0x000F000Fu) | 0x43004300u;
@@ -367,17 +359,11 @@ gemv_mma(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restrict_
       const uint4 u = ld_nc_u4(xs + 8 * v);
       xw[4 * v] = u.x; xw[4 * v + 1] = u.y; xw[4 * v + 2] = u.z; xw[4 * v + 3] = u.w;
     }
+    uint32_t frag[16];
+    build_x_fragment(xw, frag);
     uint32_t* dst = xf + (static_cast<size_t>(g) * 4 * M + L) * 16;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      // word w = j/2 covers x[32c + 8w .. +7] = xw[4w .. 4w+3]; pairs (k, k+4) with
-      // k = 2(j%2) (b0) and 2(j%2) + 1 (b1)
-      const int w = j >> 1, o = (j & 1) * 2;
-      const uint32_t lo = xw[4 * w + (o >> 1)];      // (x[8w+o], x[8w+o+1])
-      const uint32_t hi = xw[4 * w + 2 + (o >> 1)];  // (x[8w+o+4], x[8w+o+5])
-      dst[2 * j] = __byte_perm(lo, hi, 0x5410);      // (x[8w+o], x[8w+o+4])
-      dst[2 * j + 1] = __byte_perm(lo, hi, 0x7632);  // (x[8w+o+1], x[8w+o+5])
-    }
+    for (int j = 0; j < 16; ++j) dst[j] = frag[j];
   }
   __syncthreads();
 
@@ -476,23 +462,6 @@ gemv_mma(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restrict_
 // The offset is small (16 against q - Z), so the fp32 cancellation costs only a few bits.
 // The X fragments (see gemv_mma) and the per-group token sums are built once per CTA.
 // Each group's 8 MMAs run as two independent accumulator chains.
-// (a & b) | c in one 3-input logic op (both constants arrive in registers, so no second op).
-__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-// (1 + q/16) bf16 pairs of a word's codes: out[i] = (k_i, k_{i+4}) for i = 0..3.
-// mask = 0x00780078, magic = 0x3F803F80 (passed in registers by the caller).
-__device__ __forceinline__ void unpack_bf16_hi(uint32_t w, uint32_t mask, uint32_t magic,
-                                               uint32_t (&out)[4]) {
-  out[0] = and_or(w << 3, mask, magic);
-  out[1] = and_or(w >> 1, mask, magic);
-  out[2] = and_or(w >> 5, mask, magic);
-  out[3] = and_or(w >> 9, mask, magic);
-}
-
 // Shared-memory layout of gemv_mma_bulk (host and device agree through this).
 struct MmaBulkLayout {
   uint32_t xf_bytes, sx_bytes, stage_bytes, wbytes, szbytes, ring_off, bar_off, red_off, total;
@@ -606,15 +575,11 @@ gemv_mma_bulk(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __rest
       const uint4 u = ld_nc_u4(xs + 8 * v);
       xw[4 * v] = u.x; xw[4 * v + 1] = u.y; xw[4 * v + 2] = u.z; xw[4 * v + 3] = u.w;
     }
+    uint32_t frag[16];
+    build_x_fragment(xw, frag);
     uint32_t* dst = xf + (static_cast<size_t>(g) * 4 * M + Lf) * 16;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int w = j >> 1, o = (j & 1) * 2;
-      const uint32_t lo = xw[4 * w + (o >> 1)];
-      const uint32_t hi = xw[4 * w + 2 + (o >> 1)];
-      dst[2 * j] = __byte_perm(lo, hi, 0x5410);
-      dst[2 * j + 1] = __byte_perm(lo, hi, 0x7632);
-    }
+    for (int j = 0; j < 16; ++j) dst[j] = frag[j];
   }
   for (int e = threadIdx.x; e < G * 8; e += 32 * NW) {
     const int g = e >> 3, n = e & 7;
@@ -1014,6 +979,10 @@ cudaError_t launch_gemv_w8a16(const Gemv8Args& a, cudaStream_t st) {
 int gemv_max_k() { return 32 * kSlice; }
 
 cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st) {
+  if (gemv_stream_ok(a)) {
+    const cudaError_t e = launch_gemv_stream(a, sms, st);
+    if (e != cudaErrorInvalidValue) return e;
+  }
   if (mma_bulk_ok(a)) {
     cudaError_t e = cudaErrorInvalidValue;
     switch (a.M) {

@@ -41,6 +41,9 @@ struct GemvArgs {
   unsigned* status;
 };
 int gemv_max_k();
+// Streaming TMA-fed decode kernel for M <= 4, g = 128 (decode.cu).
+bool gemv_stream_ok(const GemvArgs& a);
+cudaError_t launch_gemv_stream(const GemvArgs& a, int sms, cudaStream_t st);
 cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st);
 
 // Small-M W8A16 (symmetric INT8 per output channel) on CUDA cores.

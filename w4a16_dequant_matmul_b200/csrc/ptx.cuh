@@ -127,6 +127,29 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Order this thread's earlier generic-proxy shared-memory accesses before its later
+// async-proxy ones (a bulk copy that overwrites what was just read).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Tiled TMA load of the box at coordinates (x, y) of a 2D tensor map (passed as a
+// __grid_constant__ kernel parameter) into this CTA's shared memory, completing as
+// transaction bytes on `bar`. No multicast.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Bring a tensor map (a __grid_constant__ kernel parameter) into the TMA unit's cache.
+__device__ __forceinline__ void prefetch_tensormap(const void* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
 // Programmatic dependent launch: let the next kernel on the stream start launching, and
 // wait until every prerequisite grid has completed with its memory visible.
 __device__ __forceinline__ void pdl_launch_dependents() {
