@@ -131,17 +131,28 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
 /* W4A16 matmul Y = X W_hat^T ("LLM Weight Quantization ...", "The vocabulary"):
  *   X [M, K] bf16 (ldx), packed/S/Z as produced above with group g (0 = per-tensor),
  *   Y [M, N] bf16 (ldy), fp32 accumulation.
- * Kernel choice by M: M <= 8 streams the packed weights on CUDA cores with the
- * dequantization in registers and S' factored out of each group (exact S'(q - Z));
- * larger M runs the tensor-core GEMM, which dequantizes each weight tile to bf16 in
- * shared memory (so W_hat is rounded to bfloat16 there).
- * Requires K % 128 == 0 for M > 8; K % 32 == 0 otherwise; ldx, ldy multiples of 8. */
+ * Kernel choice by M:
+ *   - M <= 8 (M = 1 only for K <= 32768): decode kernels. The packed rows stream through
+ *     shared memory (bulk copies) or registers, codes are decoded in registers (into
+ *     warp-level bf16 MMAs for g = 128 and N % 16 == 0, else packed fp32 FMAs), and S'
+ *     and Z are applied per group in fp32: the product is with the exact S'(q - Z). The
+ *     result is deterministic (fixed reduction order).
+ *   - larger M: the tcgen05/TMEM tensor-core GEMM, which dequantizes each weight tile to
+ *     bf16 in shared memory (so W_hat is rounded to bfloat16 there, then multiplied
+ *     exactly with fp32 accumulation).
+ * Requirements: K % 32 == 0; g a multiple of 32 dividing K, or 0; X 16-byte aligned and
+ * ldx % 8 == 0; packed 16-byte aligned; S, Z, Y 2-byte aligned. On the tensor-core path
+ * also K % 64 == 0 (else WQ_ERR_SHAPE), Y 16-byte aligned and ldy % 8 == 0 (else
+ * WQ_ERR_ALIGN). A launch may start before the previous kernel on the stream ends
+ * (programmatic dependent launch); it reads its inputs only after that kernel completes. */
 wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* packed,
                         const uint16_t* S, const uint16_t* Z, int64_t N, int64_t K,
                         int32_t group, uint16_t* Y, int64_t ldy, void* stream);
 
 /* W8A16 matmul with INT8 symmetric per-channel weights: codes int8 [N, K], S [N]
- * binary16; Y = X (s' q)^T, fp32 accumulation, bf16 out. Same M rules as above. */
+ * binary16; Y = X (s' q)^T, fp32 accumulation, bf16 out. M <= 8 runs on CUDA cores with
+ * the exact s' q; larger M on the tensor-core GEMM (s' q rounded to bf16). Same
+ * requirements as wq_w4a16_gemm. */
 wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t* codes,
                         const uint16_t* S, int64_t N, int64_t K, uint16_t* Y, int64_t ldy,
                         void* stream);
