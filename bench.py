@@ -9,10 +9,11 @@ Weights cycle through rotating copies totalling more than 3x the L2 cache, so ev
 launch streams its weights from HBM. Timing: CUDA graphs of the steps, CUDA events on the
 capturing stream, barrier + synchronize on both sides, max over ranks.
 
-Also reported (outside the timed step): M = 4 and 16 on the same shapes, the quantizer
-over the 70B-class weights (28672 x 8192, 8192 x 28672), the prefill GEMM
-(2048 x 4096 x 11008) when the tensor-core path is available, the oracle on the host
-cores (cpu_baseline) and the end-to-end rate through host buffers (e2e).
+Also reported (outside the timed step): M = 4, 8, 16 and 32 on the same shapes, the
+quantizer over the 70B-class weights (28672 x 8192, 8192 x 28672) and the 70B decode layer
+at M = 1, 8 and 32 on them, the prefill GEMM (2048 x 4096 x 11008) in W4A16 and in W8A16,
+the oracle on the host cores (cpu_baseline) and the end-to-end rate through host buffers
+(e2e).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -359,9 +360,9 @@ def run_gpu(args):
         us = graph_time_us(one, 4 * nsets)
         per_shape[f"{N}x{K}"] = {"us": round(us, 3), "GB/s": round(gemv_bytes(1, N, K) / us / 1e3, 1)}
 
-    # ---- secondary: M = 4, 16 on the same shapes
+    # ---- secondary: M = 4, 8, 16, 32 on the same shapes
     secondary = {}
-    for M in (4, 16):
+    for M in (4, 8, 16, 32):
         tot_b, tot_us = 0, 0.0
         for j, (N, K) in enumerate(SHAPES):
             Xm = torch.from_numpy(wq_inputs.act_bf16(M, K).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -382,8 +383,9 @@ def run_gpu(args):
         else:
             secondary[f"gemv_M{M}_GB/s"] = round(tot_b / tot_us / 1e3, 1)
 
-    # ---- secondary: quantizer over the 70B-class weights
-    qres = {}
+    # ---- secondary: quantizer over the 70B-class weights, then the 70B decode layer
+    # (M = 1, 8, 32) on the two quantized matrices, alternating (250 MB > L2)
+    qres, q70 = {}, []
     for (N, K) in wq_inputs.SHAPES_70B:
         Wt = (torch.randn(N, K, device=dev) * 0.015).to(torch.bfloat16)
         p = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
@@ -392,8 +394,24 @@ def run_gpu(args):
         us = graph_time_us(lambda: wq.wq_quantize_rtn_g128(Wt, packed=p, S=s, Z=z), 5)
         qb = N * K * 2 + N * K // 2 + 4 * N * (K // 128)
         qres[f"{N}x{K}"] = {"us": round(us, 1), "GB/s": round(qb / us / 1e3, 1)}
-        del Wt, p, s, z
+        q70.append((N, K, p, s, z))
+        del Wt
     secondary["quantizer_70b"] = qres
+    d70 = {}
+    for M in (1, 8, 32):
+        Xs = [torch.from_numpy(wq_inputs.act_bf16(M, K).view(np.int16)).view(torch.bfloat16).to(dev)
+              for (_, K, _, _, _) in q70]
+        Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (N, _, _, _, _) in q70]
+
+        def both(Xs=Xs, Ys=Ys):
+            for j, (N, K, p, s, z) in enumerate(q70):
+                wq.wq_w4a16_gemm(Xs[j], p, s, z, 128, Y=Ys[j])
+        us = graph_time_us(both, 4)
+        b70 = sum(gemv_bytes(M, N, K) for (N, K, _, _, _) in q70)
+        d70[f"M{M}"] = {"us_per_pair": round(us, 1), "GB/s": round(b70 / us / 1e3, 1),
+                        "frac": round(b70 / us / 1e3 / peaks["hbm_gbs"], 4)}
+    secondary["decode_70b"] = dict(d70, shapes="28672x8192 + 8192x28672 per step")
+    del q70
     assert wq.wq_get_status() == 0
 
     # ---- secondary: prefill GEMM (tensor cores)
@@ -409,7 +427,12 @@ def run_gpu(args):
         prefill = {"us": round(us, 1), "TFLOP/s": round(tflops, 1),
                    "peak": peaks["bf16_tflops"], "frac": round(tflops / peaks["bf16_tflops"], 4),
                    "shape": "M=2048 N=11008 K=4096"}
-        del Wt, pk, s, z, Xp, Yp
+        q8, s8, _ = wq.wq_quantize_rtn_g128(Wt, 8, P["K"], False)
+        us8 = graph_time_us(lambda: wq.wq_w8a16_gemm(Xp, q8, s8, Y=Yp), 10)
+        tf8 = 2.0 * P["M"] * P["N"] * P["K"] / us8 / 1e6
+        prefill["w8a16"] = {"us": round(us8, 1), "TFLOP/s": round(tf8, 1),
+                            "frac": round(tf8 / peaks["bf16_tflops"], 4)}
+        del Wt, pk, s, z, Xp, Yp, q8, s8
     except Exception as e:  # the tensor-core path may be missing
         prefill = f"unavailable: {e}"
     secondary["prefill"] = prefill

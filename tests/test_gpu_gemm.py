@@ -145,6 +145,39 @@ def test_stream_many_tiles_sampled(N, K, M):
     assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref) <= GATE
 
 
+@pytest.mark.parametrize("M", [8, 9, 16, 24, 32])
+@pytest.mark.parametrize("N,K", [(256, 4096), (32, 11008)])
+def test_token_block_passes(N, K, M):
+    """M with no single fast decode kernel (M = 8 at K = 11008, and 9..32) runs as passes
+    over blocks of tokens; each pass is an exact-mode decode."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + 3 * K)
+    Xb = wq_inputs.act_bf16(M, K, seed=M + 77)
+    packed, S, Z, codes, So, Zo = _quantize_both(Wb, 128)
+    X = gu.bf16_from_bits(Xb)
+    Y = wq.wq_w4a16_gemm(X, packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "exact")
+    y = gu.bf16_to_f64(Y)
+    assert oracle.gemm_gate(y, Yref) <= GATE
+    assert oracle.rel_frobenius(Yref, y) < 4e-3
+
+
+@pytest.mark.parametrize("M", [16, 32])
+def test_skinny_full_size_sampled(M):
+    """11008 x 4096 at M = 16 and 32 (the skinny decode sizes), sampled rows."""
+    N, K = 11008, 4096
+    Wb = wq_inputs.weight_bf16(N, K, 0.02)
+    Xb = wq_inputs.act_bf16(M, K, seed=5)
+    packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb))
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    rows = np.sort(np.random.default_rng(M).choice(N, 48, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    codes, So, Zo = oracle.quantize_rtn_asym(wq_inputs.bf16_bits_to_f64(Wb[rows]), 128)
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "exact")
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref) <= GATE
+
+
 @pytest.mark.parametrize("M", [1, 3, 8])
 def test_w8a16_small_m(M):
     N, K = 130, 2048

@@ -173,6 +173,11 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
                                       static_cast<cudaStream_t>(stream)));
 }
 
+// Token counts up to which the decode kernels (in passes of at most 8 tokens, at most
+// kMaxPasses of them) beat the tensor-core GEMM, whose tiles are too few for small M.
+constexpr int64_t kSkinnyMaxM = 32;
+constexpr int64_t kMaxPasses = 8;
+
 wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* packed,
                         const uint16_t* S, const uint16_t* Z, int64_t N, int64_t K,
                         int32_t group, uint16_t* Y, int64_t ldy, void* stream) {
@@ -190,9 +195,27 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int g = group ? group : (int)K;
   const int sz_row = group ? (int)(K / group) : 0;
-  if (M <= 8 && (M > 1 || K <= wq::gemv_max_k())) {
-    wq::GemvArgs a{X, ldx, packed, S, Z, (int)M, (int)N, (int)K, g, sz_row, Y, ldy, d->status};
-    return from_cuda(wq::launch_gemv_w4a16(a, d->sms, st));
+  if (M <= kSkinnyMaxM && (M > 1 || K <= wq::gemv_max_k())) {
+    // Small M: the decode kernels, in passes over blocks of tokens when the whole of M has
+    // no fast kernel (the weights come from HBM once; later passes find them in L2).
+    wq::GemvArgs a{X, ldx, packed, S, Z, (int)(M < 8 ? M : 8), (int)N, (int)K, g, sz_row, Y,
+                   ldy, d->status};
+    const int b = wq::gemv_fast_block(a);
+    if (b > 0 && (M + b - 1) / b <= kMaxPasses) {
+      for (int64_t m0 = 0; m0 < M; m0 += b) {
+        wq::GemvArgs p = a;
+        p.X = X + m0 * ldx;
+        p.Y = Y + m0 * ldy;
+        p.M = static_cast<int>(M - m0 < b ? M - m0 : b);
+        const wq_status e = from_cuda(wq::launch_gemv_w4a16(p, d->sms, st));
+        if (e != WQ_OK) return e;
+      }
+      return WQ_OK;
+    }
+    if (M <= 8) {
+      a.M = (int)M;
+      return from_cuda(wq::launch_gemv_w4a16(a, d->sms, st));
+    }
   }
   wq::TcGemmArgs a{X, ldx, packed, S, Z, nullptr, (int)M, (int)N, (int)K, g, sz_row, Y, ldy};
   return wq::launch_tc_gemm(a, d->sms, d->status, st);

@@ -451,6 +451,17 @@ cudaError_t launch_decode_m(const GemvArgs& a, int sms, cudaStream_t st) {
 
 }  // namespace
 
+bool gemv_stream_fits(const GemvArgs& a) {
+  if (a.M < 2 || a.M > 4 || a.K % 128 != 0) return false;
+  const int row_bytes = a.K / 2;
+  const int NCH = (row_bytes + kChunkMax - 1) / kChunkMax;
+  const int CK = static_cast<int>(align_up((row_bytes + NCH - 1) / NCH, 64));
+  if ((NCH - 1) * CK >= row_bytes) return false;
+  const int pitch = CK + ((64 - CK % 128) + 128) % 128;
+  const DecodeLayout base(a.M, a.K / 128, pitch, 2, 2);
+  return base.total + 128 <= kSmemBudget;
+}
+
 bool gemv_stream_ok(const GemvArgs& a) {
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   // M = 1 stays on the 32-row-tile kernel (gemv_mma_bulk), measured faster there

@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(256)
 gemv_mma(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restrict__ P,
          const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int N, int K,
          int group, int sz_row, uint16_t* __restrict__ Y, int64_t ldy) {
-  extern __shared__ __align__(16) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem[];
   const int G = K / 128;
   uint32_t* xf = reinterpret_cast<uint32_t*>(smem);                      // [G][4M][16]
   float* red = reinterpret_cast<float*>(smem + static_cast<size_t>(G) * 4 * M * 64);  // [8][16][8]
@@ -977,6 +977,25 @@ cudaError_t launch_gemv_w8a16(const Gemv8Args& a, cudaStream_t st) {
 }
 
 int gemv_max_k() { return 32 * kSlice; }
+
+// Token block b <= a.M (a.M itself if it fits, else the largest of 8, 4, 2, 1) for which a
+// bulk-fed MMA decode kernel (gemv_mma_bulk, or the streaming kernel for b = 2..4) fits
+// this shape; 0 if none.
+int gemv_fast_block(const GemvArgs& a) {
+  if (!mma_bulk_ok(a)) return 0;
+  const int half = a.K / 2;
+  const int wstride = half + ((64 - half % 128) + 128) % 128;
+  auto bulk_fits = [&](int m) {
+    return MmaBulkLayout(m, a.K, wstride, 2, kDecodeWarps, 1).total <= 220u * 1024;
+  };
+  for (int b : {a.M, 8, 4, 2, 1}) {  // the whole of M first, then blocks
+    if (b > a.M || b > 8) continue;
+    GemvArgs t = a;
+    t.M = b;
+    if (bulk_fits(b) || (b >= 2 && gemv_stream_fits(t))) return b;
+  }
+  return 0;
+}
 
 cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st) {
   if (gemv_stream_ok(a)) {
