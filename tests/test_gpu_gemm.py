@@ -145,6 +145,24 @@ def test_stream_many_tiles_sampled(N, K, M):
     assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref) <= GATE
 
 
+@pytest.mark.parametrize("N,K", [(8, 256), (100, 768), (1000, 4096), (4104, 4096), (96, 11008),
+                                 (300, 8192)])
+def test_m1_decode_shapes(N, K):
+    """M = 1 at assorted sizes: one row block, ragged row blocks, a row count just past a
+    multiple of the tile, K up to 11008; bitwise repeatable."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + 5 * K)
+    Xb = wq_inputs.act_bf16(1, K, seed=K)
+    packed, S, Z, codes, So, Zo = _quantize_both(Wb, 128)
+    X = gu.bf16_from_bits(Xb)
+    Y = wq.wq_w4a16_gemm(X, packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "exact")
+    y = gu.bf16_to_f64(Y)
+    assert oracle.gemm_gate(y, Yref) <= GATE
+    assert oracle.rel_frobenius(Yref, y) < 4e-3
+    assert torch.equal(Y, wq.wq_w4a16_gemm(X, packed, S, Z, 128))
+
+
 @pytest.mark.parametrize("M", [8, 9, 16, 24, 32])
 @pytest.mark.parametrize("N,K", [(256, 4096), (32, 11008)])
 def test_token_block_passes(N, K, M):
