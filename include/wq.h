@@ -132,7 +132,8 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
  *   X [M, K] bf16 (ldx), packed/S/Z as produced above with group g (0 = per-tensor),
  *   Y [M, N] bf16 (ldy), fp32 accumulation.
  * Kernel choice by M:
- *   - M <= 8 (M = 1 only for K <= 32768): decode kernels. The packed rows stream through
+ *   - M <= 8 (M = 1 with K > 32768 only for g = 128, K % 128 == 0, N % 16 == 0 and
+ *     16-byte aligned S, Z): decode kernels. The packed rows stream through
  *     shared memory (bulk copies) or registers, codes are decoded in registers (into
  *     warp-level bf16 MMAs for g = 128 and N % 16 == 0, else packed fp32 FMAs), and S'
  *     and Z are applied per group in fp32: the product is with the exact S'(q - Z). The

@@ -146,10 +146,12 @@ def test_stream_many_tiles_sampled(N, K, M):
 
 
 @pytest.mark.parametrize("N,K", [(8, 256), (100, 768), (1000, 4096), (4104, 4096), (96, 11008),
-                                 (300, 8192)])
+                                 (300, 8192), (48, 28672), (32, 40960)])
 def test_m1_decode_shapes(N, K):
     """M = 1 at assorted sizes: one row block, ragged row blocks, a row count just past a
-    multiple of the tile, K up to 11008; bitwise repeatable."""
+    multiple of the tile, K up to 11008, and K whose rows do not fit in shared memory whole
+    (28672, the 70B down projection, and 40960, past the register-loaded kernels): those
+    run on the streaming kernel in K chunks; bitwise repeatable."""
     Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + 5 * K)
     Xb = wq_inputs.act_bf16(1, K, seed=K)
     packed, S, Z, codes, So, Zo = _quantize_both(Wb, 128)

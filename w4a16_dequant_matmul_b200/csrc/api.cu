@@ -195,11 +195,14 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int g = group ? group : (int)K;
   const int sz_row = group ? (int)(K / group) : 0;
-  if (M <= kSkinnyMaxM && (M > 1 || K <= wq::gemv_max_k())) {
+  wq::GemvArgs a{X, ldx, packed, S, Z, (int)(M < 8 ? M : 8), (int)N, (int)K, g, sz_row, Y,
+                 ldy, d->status};
+  // M = 1 beyond the register-loaded kernels' K only where the streaming kernel takes it
+  if (M <= kSkinnyMaxM &&
+      (M > 1 || K <= wq::gemv_max_k() || wq::gemv_tma_ok(a) ||
+       (wq::gemv_stream_ok(a) && wq::gemv_stream_fits(a)))) {
     // Small M: the decode kernels, in passes over blocks of tokens when the whole of M has
     // no fast kernel (the weights come from HBM once; later passes find them in L2).
-    wq::GemvArgs a{X, ldx, packed, S, Z, (int)(M < 8 ? M : 8), (int)N, (int)K, g, sz_row, Y,
-                   ldy, d->status};
     const int b = wq::gemv_fast_block(a);
     if (b > 0 && (M + b - 1) / b <= kMaxPasses) {
       for (int64_t m0 = 0; m0 < M; m0 += b) {
@@ -217,8 +220,8 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
       return from_cuda(wq::launch_gemv_w4a16(a, d->sms, st));
     }
   }
-  wq::TcGemmArgs a{X, ldx, packed, S, Z, nullptr, (int)M, (int)N, (int)K, g, sz_row, Y, ldy};
-  return wq::launch_tc_gemm(a, d->sms, d->status, st);
+  wq::TcGemmArgs t{X, ldx, packed, S, Z, nullptr, (int)M, (int)N, (int)K, g, sz_row, Y, ldy};
+  return wq::launch_tc_gemm(t, d->sms, d->status, st);
 }
 
 wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t* codes,

@@ -288,9 +288,7 @@ gemv_decode(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restri
   const uint32_t xf_lane = base_s + L.xf + xn * (G * 256) + c * 64;
   const uint32_t ring_lane = base_s + L.ring + r * pitch + 16 * c;
   uint32_t kMask = 0x00780078u, kMagic = 0x3F803F80u;  // register operands of the LOP3
-  uint32_t kMul[4] = {8u, 1u << 31, 1u << 27, 1u << 23};
-  asm volatile("" : "+r"(kMask), "+r"(kMagic), "+r"(kMul[0]), "+r"(kMul[1]), "+r"(kMul[2]),
-               "+r"(kMul[3]));
+  asm volatile("" : "+r"(kMask), "+r"(kMagic));
   const int gpc = CK / 64;  // groups per full chunk
   // One group (128 codes) of RT consecutive 16-row tiles: the X fragments are read once for
   // all of them. wst[t] / prep[t]: this lane's row in the chunk stage / S'Z slot of tile t.
@@ -315,8 +313,8 @@ gemv_decode(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restri
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         uint32_t pa[4], pb[4];
-        unpack_bf16_hi_imad(wr0[w], kMask, kMagic, kMul, pa);
-        unpack_bf16_hi_imad(wr1[w], kMask, kMagic, kMul, pb);
+        unpack_bf16_hi(wr0[w], kMask, kMagic, pa);
+        unpack_bf16_hi(wr1[w], kMask, kMagic, pb);
         const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
         const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
         mma_bf16_16816(d[(w & 1) * 2], a0, bw[4 * w], bw[4 * w + 1]);
@@ -452,7 +450,7 @@ cudaError_t launch_decode_m(const GemvArgs& a, int sms, cudaStream_t st) {
 }  // namespace
 
 bool gemv_stream_fits(const GemvArgs& a) {
-  if (a.M < 2 || a.M > 4 || a.K % 128 != 0) return false;
+  if (a.M < 1 || a.M > 4 || a.K % 128 != 0) return false;
   const int row_bytes = a.K / 2;
   const int NCH = (row_bytes + kChunkMax - 1) / kChunkMax;
   const int CK = static_cast<int>(align_up((row_bytes + NCH - 1) / NCH, 64));
@@ -464,8 +462,7 @@ bool gemv_stream_fits(const GemvArgs& a) {
 
 bool gemv_stream_ok(const GemvArgs& a) {
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  // M = 1 stays on the 32-row-tile kernel (gemv_mma_bulk), measured faster there
-  return a.M >= 2 && a.M <= 4 && a.K % 128 == 0 && a.sz_row > 0 && a.group == 128 &&
+  return a.M >= 1 && a.M <= 4 && a.K % 128 == 0 && a.sz_row > 0 && a.group == 128 &&
          a.N % 16 == 0 && (a.ldx % 8) == 0 && al16(a.X) && al16(a.P) && al16(a.S) && al16(a.Z);
 }
 

@@ -1,0 +1,411 @@
+// Small-M W4A16 matmul (decode) on 32-row weight tiles fed by TMA: Y = X W_hat^T for
+// M <= 4 tokens, group size 128, N a multiple of 32.
+// ("LLM Weight Quantization - GPTQ, AWQ, SmoothQuant, FP8 & INT4/INT8 Trade-offs",
+// "The vocabulary" and the decode discussion: 4-bit weights dequantized inside the kernel;
+// at decode the matmul is bound by the bytes of weights read from memory.)
+//
+// Work: tiles of 32 weight rows; a CTA owns a contiguous, balanced range of them. A tile
+// streams in chunks of 8 groups (1024 k): one TMA box of 64 bytes x 32 rows x 8 groups
+// (16 KB) that lands as [group][row][64 B], so the two rows a quarter-warp reads sit 64
+// bytes apart and its 16-byte loads cover all 32 banks. The tile's S' and Z (32 x G each,
+// contiguous in HBM) arrive by two bulk copies into a slot of their own.
+//
+// A CTA uses less than half of an SM's shared memory and registers, so the next launch on
+// the stream can take the other half while this one finishes. Each CTA lets the next
+// launch start at once (programmatic dependent launch), warms L2 with its first chunks and
+// S'/Z (hints, which are safe before the dependency wait), and then waits for the previous
+// kernel before it copies or writes anything.
+//
+// Warp roles:
+//   producer  one lane: X (one bulk copy per token), then per tile the S'/Z copies and the
+//             chunk boxes into a ring of 16 KB stages.
+//   consumers 8 warps. Every warp takes every chunk and its share of the chunk's groups, so
+//             each warp waits for every fill of every stage in order (the parity waits
+//             cannot alias). Per group a warp reads the X fragments once and multiplies both
+//             16-row halves of the tile: codes decoded to bf16 (1 + q/16), eight m16n8k16
+//             MMAs per half in four accumulator chains, and with D = sum x (1 + q/16),
+//               acc += S' (16 D - (16 + Z) sum x).
+//   epilogue  sums the 8 warps' partials of a tile in warp order (deterministic) and writes
+//             Y in bf16.
+// Every wait is bounded (2 s): on a timeout the kernel records kStTimeout, the producer waits
+// (bounded) for the copies it issued, and all warps return.
+#include "common.cuh"
+#include "kernels.h"
+#include "mma_frag.cuh"
+#include "ptx.cuh"
+#include "tma_host.h"
+
+namespace wq {
+namespace {
+
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kNW = 16;                          // consumer warps
+constexpr int kTR = 32;                          // weight rows per tile
+constexpr int kMaxCG = 32;                       // groups per chunk, at most (64 KB)
+constexpr int kSzSlots = 2;                      // tiles of S'/Z in flight
+constexpr int kPartSlots = 2;                    // tiles between consumers and epilogue
+constexpr int kMaxStages = 8;
+constexpr int kThreads = 32 * (kNW + 2);
+constexpr uint32_t kSmemBudget = 227 * 1024;     // one CTA per SM
+constexpr uint64_t kPrefetchBudget = 48ull << 20;  // L2 warm-up per launch, all CTAs
+constexpr uint32_t kSlack = 128;                 // aligning the dynamic base
+
+__host__ __device__ constexpr uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+// Shared-memory layout (byte offsets from a 128-aligned base; host and device agree).
+struct TmaLayout {
+  uint32_t xf, xsp, sx, sz, sz_slot, part, part_slot, ring, bar, total;
+  __host__ __device__ TmaLayout(int M, int G, int NS, int CG) {
+    const uint32_t MR = M < 2 ? 2 : M;
+    xf = 0;                                  // [M][G][4][16] u32 X fragments
+    xsp = xf + G * 4u * M * 64;              // [M][G][4] f32 partial sums of x
+    sx = xsp + G * 4u * M * 4;               // [G][8] f32 sums of x per token
+    sz = align_up(sx + G * 32u, 128);
+    sz_slot = align_up(128u * G, 128);       // S' [32][G] u16, then Z [32][G] u16
+    part = sz + kSzSlots * sz_slot;
+    part_slot = kNW * kTR * MR * 4;          // [16 warps][32 rows][MR] f32
+    ring = align_up(part + kPartSlots * part_slot, 128);
+    bar = ring + NS * (kTR * 64u * CG);
+    total = bar + (2u * NS + 2u * kSzSlots + 2u * kPartSlots + 1u) * 8;
+  }
+};
+
+template <int M>
+__global__ void __launch_bounds__(kThreads, 1)
+gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X, int64_t ldx,
+         const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int N, int K, int NS,
+         int CG, int prefetch_tiles, uint16_t* __restrict__ Y, int64_t ldy, unsigned* status) {
+  constexpr int MR = M < 2 ? 2 : M;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+  const uint32_t base_s = smem_u32(smem);
+  const int G = K / 128;
+  const int NCH = (G + CG - 1) / CG;
+  const uint32_t stage = kTR * 64u * CG;  // bytes of one chunk
+  const TmaLayout L(M, G, NS, CG);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
+  uint64_t* empty = full + NS;
+  uint64_t* szfull = empty + NS;
+  uint64_t* szempty = szfull + kSzSlots;
+  uint64_t* tdone = szempty + kSzSlots;
+  uint64_t* pempty = tdone + kPartSlots;
+  uint64_t* xfull = pempty + kPartSlots;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ntiles = N / kTR;
+  const int t_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * ntiles / gridDim.x);
+  const int t_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * ntiles / gridDim.x);
+  const int my_tiles = t_end - t_begin;
+  const uint32_t szbytes = 64u * G;  // one of S', Z for a tile
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kNW);
+    }
+    for (int i = 0; i < kSzSlots; ++i) {
+      mbar_init(&szfull[i], 1);
+      mbar_init(&szempty[i], kNW);
+    }
+    for (int i = 0; i < kPartSlots; ++i) {
+      mbar_init(&tdone[i], kNW);
+      mbar_init(&pempty[i], 1);
+    }
+    mbar_init(xfull, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  if (warp == kNW && lane == 0) {
+    // warm L2 with this CTA's first tiles, codes and S'/Z (hints only): the reads then run
+    // at the full HBM rate, ahead of the ring
+    prefetch_tensormap(&tmW);
+    for (int t = t_begin; t < t_end && t < t_begin + prefetch_tiles; ++t) {
+      prefetch_l2_bulk(S + static_cast<int64_t>(t) * kTR * G, szbytes);
+      prefetch_l2_bulk(Zp + static_cast<int64_t>(t) * kTR * G, szbytes);
+      for (int ch = 0; ch < NCH; ++ch) tma_prefetch_3d(&tmW, 0, t * kTR, ch * CG);
+    }
+  }
+  pdl_wait();
+
+  if (warp == kNW) {  // ---------------------------------------------------------- producer
+    if (lane != 0) return;
+    mbar_arrive_expect_tx(xfull, static_cast<uint32_t>(M) * K * 2);
+    for (int n = 0; n < M; ++n)
+      bulk_g2s(smem + L.xf + static_cast<uint32_t>(n) * K * 2, X + n * ldx, K * 2u, xfull);
+    int i = 0, tl = 0;
+    bool ok = true;
+    for (; tl < my_tiles && ok; ++tl) {
+      const int tile = t_begin + tl, ss = tl % kSzSlots;
+      if (tl >= kSzSlots &&
+          !mbar_wait_spin_bounded(&szempty[ss], ((tl / kSzSlots) - 1) & 1u, kWaitNs)) {
+        set_status(status, kStTimeout);
+        break;
+      }
+      uint8_t* sd = smem + L.sz + ss * L.sz_slot;
+      mbar_arrive_expect_tx(&szfull[ss], 2u * szbytes);
+      bulk_g2s(sd, S + static_cast<int64_t>(tile) * kTR * G, szbytes, &szfull[ss]);
+      bulk_g2s(sd + szbytes, Zp + static_cast<int64_t>(tile) * kTR * G, szbytes, &szfull[ss]);
+      for (int ch = 0; ch < NCH; ++ch, ++i) {
+        const int st = i % NS;
+        const uint32_t use = i / NS;
+        if (use > 0 && !mbar_wait_spin_bounded(&empty[st], (use - 1) & 1u, kWaitNs)) {
+          set_status(status, kStTimeout);
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[st], stage);
+        tma_load_3d(smem + L.ring + st * stage, &tmW, 0, tile * kTR, ch * CG, &full[st]);
+      }
+    }
+    // never leave the CTA with copies in flight
+    for (int st = 0; st < NS && st < i; ++st)
+      if (!mbar_wait_spin_bounded(&full[st], ((i - 1 - st) / NS) & 1u, kWaitNs))
+        set_status(status, kStTimeout);
+    for (int ss = 0; ss < kSzSlots && ss < tl; ++ss)
+      if (!mbar_wait_spin_bounded(&szfull[ss], ((tl - 1 - ss) / kSzSlots) & 1u, kWaitNs))
+        set_status(status, kStTimeout);
+    if (!mbar_wait_spin_bounded(xfull, 0, kWaitNs)) set_status(status, kStTimeout);
+    return;
+  }
+
+  if (warp == kNW + 1) {  // ------------------------------------------------------ epilogue
+    for (int tl = 0; tl < my_tiles; ++tl) {
+      const int ps = tl % kPartSlots;
+      if (!mbar_wait_spin_bounded(&tdone[ps], (tl / kPartSlots) & 1u, kWaitNs)) {
+        set_status(status, kStTimeout);
+        return;
+      }
+      const float* part = reinterpret_cast<const float*>(smem + L.part + ps * L.part_slot);
+      const int tile = t_begin + tl;
+      for (int e = lane; e < kTR * M; e += 32) {
+        const int row = e / M, tok = e - (e / M) * M;
+        float t = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) t += part[(w * kTR + row) * MR + tok];
+        __nv_bfloat16 hv = __float2bfloat16_rn(t);
+        Y[tok * ldy + tile * kTR + row] = *reinterpret_cast<uint16_t*>(&hv);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pempty[ps]);
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------------- consumer warps
+  // X (landed in natural order) -> fragment order in place, 64 bytes (32 values of one
+  // token, one quarter of a group) per thread, and per-group token sums, each formed from
+  // four partial sums of 32 values in a fixed order.
+  float* xsp = reinterpret_cast<float*>(smem + L.xsp);
+  float* sxs = reinterpret_cast<float*>(smem + L.sx);
+  if (!mbar_wait_spin_bounded(xfull, 0, kWaitNs)) {
+    set_status(status, kStTimeout);
+    return;
+  }
+  for (int e = threadIdx.x; e < M * G * 4; e += 32 * kNW) {  // e = (n * G + g) * 4 + c
+    const uint32_t blk = base_s + L.xf + e * 64;
+    uint32_t xw[16];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 u = lds128(blk + 16 * v);
+      xw[4 * v] = u.x; xw[4 * v + 1] = u.y; xw[4 * v + 2] = u.z; xw[4 * v + 3] = u.w;
+    }
+    uint32_t frag[16];
+    build_x_fragment(xw, frag);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      sts128(blk + 16 * j, make_uint4(frag[4 * j], frag[4 * j + 1], frag[4 * j + 2], frag[4 * j + 3]));
+    float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int v = 0; v < 16; ++v) ps[v & 3] += bf16_lo(xw[v]) + bf16_hi(xw[v]);
+    xsp[e] = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+  }
+  named_barrier(1, 32 * kNW);
+  for (int e = threadIdx.x; e < G * 8; e += 32 * kNW) {
+    const int g = e >> 3, n = e & 7;
+    float t = 0.0f;
+    if (n < M) {
+      const float* q = xsp + (n * G + g) * 4;
+      t = (q[0] + q[1]) + (q[2] + q[3]);
+    }
+    sxs[e] = t;
+  }
+  named_barrier(1, 32 * kNW);
+
+  const int r = lane >> 2, c = lane & 3;
+  const int t0 = 2 * c, t1 = 2 * c + 1;
+  // lanes whose token column is >= M read a duplicate fragment: their columns are never
+  // stored, and the loads stay uniform
+  const int xn = (lane >> 2) % M;
+  const uint32_t xf_lane = base_s + L.xf + xn * (G * 256) + c * 64;
+  const uint32_t ring_lane = base_s + L.ring + r * 64 + 16 * c;
+  uint32_t kMask = 0x00780078u, kMagic = 0x3F803F80u;  // register operands of the LOP3
+  asm volatile("" : "+r"(kMask), "+r"(kMagic));
+  int i = 0;
+  for (int tl = 0; tl < my_tiles; ++tl) {
+    const int ss = tl % kSzSlots, ps = tl % kPartSlots;
+    const uint32_t sb = base_s + L.sz + ss * L.sz_slot, zb = sb + szbytes;
+    float acc[2][4] = {};
+    for (int ch = 0; ch < NCH; ++ch, ++i) {
+      const int st = i % NS;
+      bool ok = mbar_wait_spin_bounded(&full[st], (i / NS) & 1u, kWaitNs);
+      if (ok && ch == 0) ok = mbar_wait_spin_bounded(&szfull[ss], (tl / kSzSlots) & 1u, kWaitNs);
+      if (!ok) {
+        set_status(status, kStTimeout);
+        return;
+      }
+      const uint32_t wst = ring_lane + st * stage;
+      const int g0 = ch * CG;
+      const int gn = min(CG, G - g0);
+      const int qa = (warp * gn) / kNW, qb = ((warp + 1) * gn) / kNW;
+      for (int q = qa; q < qb; ++q) {
+        const int g = g0 + q;
+        const uint32_t xs = xf_lane + g * 256;
+        const uint4 xb0 = lds128(xs), xb1 = lds128(xs + 16), xb2 = lds128(xs + 32),
+                    xb3 = lds128(xs + 48);
+        const uint32_t bw[16] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w,
+                                 xb2.x, xb2.y, xb2.z, xb2.w, xb3.x, xb3.y, xb3.z, xb3.w};
+        const float sx0 = sxs[g * 8 + t0];
+        [[maybe_unused]] const float sx1 = M > 1 ? sxs[g * 8 + t1] : 0.0f;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t wa = wst + q * (kTR * 64) + t * (16 * 64);
+          const uint4 ca = lds128(wa);
+          const uint4 cb = lds128(wa + 8 * 64);
+          const uint32_t wr0[4] = {ca.x, ca.y, ca.z, ca.w};
+          const uint32_t wr1[4] = {cb.x, cb.y, cb.z, cb.w};
+          float d[4][4] = {};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint32_t pa[4], pb[4];
+            unpack_bf16_hi(wr0[w], kMask, kMagic, pa);
+            unpack_bf16_hi(wr1[w], kMask, kMagic, pb);
+            const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
+            const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
+            mma_bf16_16816(d[(w & 1) * 2], a0, bw[4 * w], bw[4 * w + 1]);
+            mma_bf16_16816(d[(w & 1) * 2 + 1], a1, bw[4 * w + 2], bw[4 * w + 3]);
+          }
+          const int ra = 16 * t + r, rb = ra + 8;
+          const float s0 = f16_bits_to_f32(lds16(sb + (ra * G + g) * 2));
+          const float z0 = f16_bits_to_f32(lds16(zb + (ra * G + g) * 2));
+          const float s1 = f16_bits_to_f32(lds16(sb + (rb * G + g) * 2));
+          const float z1 = f16_bits_to_f32(lds16(zb + (rb * G + g) * 2));
+          const float e0 = (d[0][0] + d[2][0]) + (d[1][0] + d[3][0]);
+          const float e2 = (d[0][2] + d[2][2]) + (d[1][2] + d[3][2]);
+          acc[t][0] = fmaf(s0, fmaf(16.0f, e0, -(16.0f + z0) * sx0), acc[t][0]);
+          acc[t][2] = fmaf(s1, fmaf(16.0f, e2, -(16.0f + z1) * sx0), acc[t][2]);
+          if constexpr (M > 1) {
+            const float e1 = (d[0][1] + d[2][1]) + (d[1][1] + d[3][1]);
+            const float e3 = (d[0][3] + d[2][3]) + (d[1][3] + d[3][3]);
+            acc[t][1] = fmaf(s0, fmaf(16.0f, e1, -(16.0f + z0) * sx1), acc[t][1]);
+            acc[t][3] = fmaf(s1, fmaf(16.0f, e3, -(16.0f + z1) * sx1), acc[t][3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    if (lane == 0) mbar_arrive(&szempty[ss]);
+    if (tl >= kPartSlots &&
+        !mbar_wait_spin_bounded(&pempty[ps], ((tl / kPartSlots) - 1) & 1u, kWaitNs)) {
+      set_status(status, kStTimeout);
+      return;
+    }
+    float* part = reinterpret_cast<float*>(smem + L.part + ps * L.part_slot) + warp * kTR * MR;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int ra = 16 * t + r, rb = ra + 8;
+      if (t0 < M) {
+        part[ra * MR + t0] = acc[t][0];
+        part[rb * MR + t0] = acc[t][2];
+      }
+      if constexpr (M > 1) {
+        if (t1 < M) {
+          part[ra * MR + t1] = acc[t][1];
+          part[rb * MR + t1] = acc[t][3];
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tdone[ps]);
+  }
+}
+
+// Chunk size (groups) and ring depth for this shape: the largest chunk of 32, 16 or 8 groups
+// whose ring has at least two stages in shared memory; NS = 0 if none fits.
+struct TmaCfg {
+  int CG, NS;
+};
+TmaCfg tma_config(int M, int G) {
+  const uint32_t fixed = TmaLayout(M, G, 0, 8).total + kSlack;
+  for (int cg : {kMaxCG, 16, 8}) {
+    if (fixed > kSmemBudget) break;
+    int ns = static_cast<int>((kSmemBudget - fixed) / (kTR * 64u * cg + 16));
+    if (ns > kMaxStages) ns = kMaxStages;
+    if (ns >= 2) return {cg, ns};
+  }
+  return {8, 0};
+}
+
+template <int M>
+cudaError_t launch_tma_m(const GemvArgs& a, int sms, cudaStream_t st) {
+  const int G = a.K / 128;
+  const int ntiles = a.N / kTR;
+  if (ntiles == 0) return cudaSuccess;
+  const TmaCfg c = tma_config(M, G);
+  if (c.NS == 0) return cudaErrorInvalidValue;
+  CUtensorMap map;
+  // codes as [G groups][N rows][64 bytes]: boxes of CG groups x 32 rows x 64 bytes
+  const uint64_t dims[3] = {64, static_cast<uint64_t>(a.N), static_cast<uint64_t>(G)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(a.K / 2), 64};
+  const uint32_t box[3] = {64, kTR, static_cast<uint32_t>(c.CG)};
+  if (!make_map_3d(&map, a.P, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+    return cudaErrorInvalidValue;
+  const size_t smem = TmaLayout(M, G, c.NS, c.CG).total + kSlack;
+  auto kern = gemv_tma<M>;
+  static bool attr[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr[dev & 63]) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(kSmemBudget));
+    if (e != cudaSuccess) return e;
+    attr[dev & 63] = true;
+  }
+  const int grid = ntiles < sms ? ntiles : sms;
+  const uint64_t tile_bytes = static_cast<uint64_t>(kTR) * (a.K / 2 + 4 * G);
+  const int prefetch_tiles = static_cast<int>(kPrefetchBudget / grid / tile_bytes);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map, a.X, a.ldx, a.S, a.Z, a.N, a.K, c.NS, c.CG,
+                            prefetch_tiles, a.Y, a.ldy, a.status);
+}
+
+}  // namespace
+
+bool gemv_tma_ok(const GemvArgs& a) {
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  return a.M >= 1 && a.M <= 4 && a.K % 128 == 0 && a.group == 128 && a.sz_row == a.K / 128 &&
+         a.N % kTR == 0 && (a.ldx % 8) == 0 && al16(a.X) && al16(a.P) && al16(a.S) &&
+         al16(a.Z) && tma_config(a.M, a.K / 128).NS > 0;
+}
+
+cudaError_t launch_gemv_tma(const GemvArgs& a, int sms, cudaStream_t st) {
+  switch (a.M) {
+    case 1: return launch_tma_m<1>(a, sms, st);
+    case 2: return launch_tma_m<2>(a, sms, st);
+    case 3: return launch_tma_m<3>(a, sms, st);
+    case 4: return launch_tma_m<4>(a, sms, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace wq

@@ -44,6 +44,9 @@ int gemv_max_k();
 // Streaming TMA-fed decode kernel for M <= 4, g = 128 (decode.cu).
 bool gemv_stream_ok(const GemvArgs& a);
 bool gemv_stream_fits(const GemvArgs& a);
+// 32-row-tile TMA-fed decode kernel for M <= 4, g = 128, N % 32 == 0 (gemv_tma.cu).
+bool gemv_tma_ok(const GemvArgs& a);
+cudaError_t launch_gemv_tma(const GemvArgs& a, int sms, cudaStream_t st);
 // Largest token block (8, 4, 2 or 1, at most a.M) with a fast decode kernel; 0 if none.
 int gemv_fast_block(const GemvArgs& a);
 cudaError_t launch_gemv_stream(const GemvArgs& a, int sms, cudaStream_t st);

@@ -43,4 +43,22 @@ inline bool make_map_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint6
   return r == CUDA_SUCCESS;
 }
 
+// 3D tiled map with arbitrary byte strides for dimensions 1 and 2 (dimension 0 is dense);
+// boxes land densely in shared memory as [box2][box1][box0]. Returns false if the driver
+// rejects the description.
+inline bool make_map_3d(CUtensorMap* map, const void* ptr, const uint64_t (&dims)[3],
+                        const uint64_t (&stride_bytes)[2], const uint32_t (&box)[3],
+                        CUtensorMapDataType dtype) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t s[2] = {stride_bytes[0], stride_bytes[1]};
+  const cuuint32_t b[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, dtype, 3, const_cast<void*>(ptr), d, s, b, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace wq
