@@ -132,12 +132,15 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
  *   X [M, K] bf16 (ldx), packed/S/Z as produced above with group g (0 = per-tensor),
  *   Y [M, N] bf16 (ldy), fp32 accumulation.
  * Kernel choice by M:
- *   - M <= 8 (M = 1 with K > 32768 only for g = 128, K % 128 == 0, N % 16 == 0 and
- *     16-byte aligned S, Z): decode kernels. The packed rows stream through
- *     shared memory (bulk copies) or registers, codes are decoded in registers (into
- *     warp-level bf16 MMAs for g = 128 and N % 16 == 0, else packed fp32 FMAs), and S'
- *     and Z are applied per group in fp32: the product is with the exact S'(q - Z). The
- *     result is deterministic (fixed reduction order).
+ *   - M <= 32: decode kernels, for M > 8 in passes over blocks of at most 8 tokens (when
+ *     some block size needs at most 8 passes; else the tensor-core GEMM). The packed rows
+ *     stream through shared memory (bulk copies or TMA boxes) or registers, codes are
+ *     decoded in registers (into warp-level bf16 MMAs for g = 128 and N % 16 == 0, else
+ *     packed fp32 FMAs), and S' and Z are applied per group in fp32: the product is with
+ *     the exact S'(q - Z). The result is deterministic (fixed reduction order). M = 1 with
+ *     K > 32768 stays on a decode kernel only where a streaming one takes the shape (g = 128,
+ *     K % 128 == 0, N % 32 == 0 or N % 16 == 0, 16-byte aligned X, S, Z, and X plus one
+ *     tile's S' and Z within shared memory); otherwise it runs on the tensor-core GEMM.
  *   - larger M: the tcgen05/TMEM tensor-core GEMM, which dequantizes each weight tile to
  *     bf16 in shared memory (so W_hat is rounded to bfloat16 there, then multiplied
  *     exactly with fp32 accumulation).
@@ -145,7 +148,9 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
  * ldx % 8 == 0; packed 16-byte aligned; S, Z, Y 2-byte aligned. On the tensor-core path
  * also K % 64 == 0 (else WQ_ERR_SHAPE), Y 16-byte aligned and ldy % 8 == 0 (else
  * WQ_ERR_ALIGN). A launch may start before the previous kernel on the stream ends
- * (programmatic dependent launch); it reads its inputs only after that kernel completes. */
+ * (programmatic dependent launch); it reads its inputs only after that kernel completes
+ * (before that it may only issue L2 prefetch hints for the weights, which cannot return
+ * stale data). */
 wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* packed,
                         const uint16_t* S, const uint16_t* Z, int64_t N, int64_t K,
                         int32_t group, uint16_t* Y, int64_t ldy, void* stream);

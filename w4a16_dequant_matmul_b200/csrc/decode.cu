@@ -19,7 +19,7 @@
 //             for a consumer lane.
 //   consumers 8 warps. Every warp takes every chunk and a fixed share of its groups, so each
 //             warp consumes each stage's fills in order (parity waits cannot alias). Codes
-//             are decoded to bf16 (1 + q/16, one multiply and one 3-input logic op per two
+//             are decoded to bf16 (1 + q/16, one shift and one 3-input logic op per two
 //             codes) and multiplied with eight m16n8k16 MMAs per group (four independent
 //             accumulator chains) against X fragments in shared memory (X arrives by one
 //             bulk copy per token and is permuted into fragment order in place); per group,

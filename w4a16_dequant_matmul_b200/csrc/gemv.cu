@@ -979,8 +979,8 @@ cudaError_t launch_gemv_w8a16(const Gemv8Args& a, cudaStream_t st) {
 int gemv_max_k() { return 32 * kSlice; }
 
 // Token block b <= a.M (a.M itself if it fits, else the largest of 8, 4, 2, 1) for which a
-// bulk-fed MMA decode kernel (gemv_mma_bulk, or the streaming kernel for b = 1..4) fits
-// this shape; 0 if none.
+// bulk-fed MMA decode kernel (gemv_mma_bulk, or for b <= 4 one of the streaming kernels)
+// fits this shape; 0 if none.
 int gemv_fast_block(const GemvArgs& a) {
   if (!mma_bulk_ok(a)) return 0;
   const int half = a.K / 2;
@@ -992,7 +992,7 @@ int gemv_fast_block(const GemvArgs& a) {
     if (b > a.M || b > 8) continue;
     GemvArgs t = a;
     t.M = b;
-    if (bulk_fits(b) || gemv_stream_fits(t) || (b == 1 && gemv_tma_ok(t))) return b;
+    if (bulk_fits(b) || gemv_stream_fits(t) || gemv_tma_ok(t)) return b;
   }
   return 0;
 }
@@ -1005,11 +1005,11 @@ static bool mma_bulk_rt2_fits(const GemvArgs& a) {
 }
 
 cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st) {
-  // M = 1: the bulk-copy kernel on whole 32-row tiles where two of them fit in shared memory
-  // (short rows: measured fastest there), else the TMA-fed kernel that streams 32-row tiles
-  // in K chunks (N % 32 == 0), then the bulk-copy kernel on 16-row tiles, then the streaming
-  // kernel (K in chunks, any K); M = 2..4: the streaming kernel first.
-  if (a.M == 1 && !(mma_bulk_ok(a) && mma_bulk_rt2_fits(a)) && gemv_tma_ok(a)) {
+  // M <= 4 with long rows (two whole 32-row tiles do not fit the bulk-copy kernel's shared
+  // memory): the TMA-fed kernel that streams 32-row tiles in K chunks (N % 32 == 0).
+  // Otherwise M = 1: the bulk-copy kernel (whole rows; measured fastest for short rows);
+  // M = 2..4: the streaming kernel on 16-row tiles.
+  if (a.M <= 4 && !(mma_bulk_ok(a) && mma_bulk_rt2_fits(a)) && gemv_tma_ok(a)) {
     const cudaError_t e = launch_gemv_tma(a, sms, st);
     if (e != cudaErrorInvalidValue) return e;
   }

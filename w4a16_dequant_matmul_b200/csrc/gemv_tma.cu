@@ -1,31 +1,28 @@
 // Small-M W4A16 matmul (decode) on 32-row weight tiles fed by TMA: Y = X W_hat^T for
-// M <= 4 tokens, group size 128, N a multiple of 32.
+// M <= 4 tokens, group size 128, N a multiple of 32. Used where a 32-row tile of whole rows is
+// too large to double-buffer in shared memory (long rows, K above about 6K).
 // ("LLM Weight Quantization - GPTQ, AWQ, SmoothQuant, FP8 & INT4/INT8 Trade-offs",
 // "The vocabulary" and the decode discussion: 4-bit weights dequantized inside the kernel;
 // at decode the matmul is bound by the bytes of weights read from memory.)
 //
-// Work: tiles of 32 weight rows; a CTA owns a contiguous, balanced range of them. A tile
-// streams in chunks of 8 groups (1024 k): one TMA box of 64 bytes x 32 rows x 8 groups
-// (16 KB) that lands as [group][row][64 B], so the two rows a quarter-warp reads sit 64
-// bytes apart and its 16-byte loads cover all 32 banks. The tile's S' and Z (32 x G each,
-// contiguous in HBM) arrive by two bulk copies into a slot of their own.
-//
-// A CTA uses less than half of an SM's shared memory and registers, so the next launch on
-// the stream can take the other half while this one finishes. Each CTA lets the next
-// launch start at once (programmatic dependent launch), warms L2 with its first chunks and
-// S'/Z (hints, which are safe before the dependency wait), and then waits for the previous
-// kernel before it copies or writes anything.
+// Work: tiles of 32 weight rows; a CTA (one per SM) owns a contiguous, balanced range of them.
+// A tile streams in chunks of CG = 32, 16 or 8 groups (the largest whose ring has two stages):
+// one TMA box of 64 bytes x 32 rows x CG groups that lands as [group][row][64 B], so the two
+// rows a quarter-warp reads sit 64 bytes apart and its 16-byte loads cover all 32 banks. The
+// tile's S' and Z (32 x G each, contiguous in HBM) arrive by two bulk copies into a slot of
+// their own. Before it waits for the previous kernel (programmatic dependent launch), each CTA
+// warms L2 with its first tiles (codes and S'/Z; hints only, so safe before the wait).
 //
 // Warp roles:
 //   producer  one lane: X (one bulk copy per token), then per tile the S'/Z copies and the
-//             chunk boxes into a ring of 16 KB stages.
-//   consumers 8 warps. Every warp takes every chunk and its share of the chunk's groups, so
+//             chunk boxes into the stage ring.
+//   consumers 16 warps. Every warp takes every chunk and its share of the chunk's groups, so
 //             each warp waits for every fill of every stage in order (the parity waits
 //             cannot alias). Per group a warp reads the X fragments once and multiplies both
 //             16-row halves of the tile: codes decoded to bf16 (1 + q/16), eight m16n8k16
 //             MMAs per half in four accumulator chains, and with D = sum x (1 + q/16),
 //               acc += S' (16 D - (16 + Z) sum x).
-//   epilogue  sums the 8 warps' partials of a tile in warp order (deterministic) and writes
+//   epilogue  sums the 16 warps' partials of a tile in warp order (deterministic) and writes
 //             Y in bf16.
 // Every wait is bounded (2 s): on a timeout the kernel records kStTimeout, the producer waits
 // (bounded) for the copies it issued, and all warps return.

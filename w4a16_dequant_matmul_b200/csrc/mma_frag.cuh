@@ -41,18 +41,6 @@ __device__ __forceinline__ void unpack_bf16_hi(uint32_t w, uint32_t mask, uint32
   out[3] = and_or(w >> 9, mask, magic);
 }
 
-// The same decode with the shifts done as integer multiplies on the FMA pipe (w * 8, and
-// the high word of w * 2^31, 2^27, 2^23 for w >> 1, 5, 9), leaving only the four logic
-// ops on the ALU pipe. k = {8, 2^31, 2^27, 2^23} arrive in registers, so the compiler
-// keeps the multiplies.
-__device__ __forceinline__ void unpack_bf16_hi_imad(uint32_t w, uint32_t mask, uint32_t magic,
-                                                    const uint32_t (&k)[4], uint32_t (&out)[4]) {
-  out[0] = and_or(w * k[0], mask, magic);
-  out[1] = and_or(__umulhi(w, k[1]), mask, magic);
-  out[2] = and_or(__umulhi(w, k[2]), mask, magic);
-  out[3] = and_or(__umulhi(w, k[3]), mask, magic);
-}
-
 // B fragments of 32 consecutive bf16 values of X (xw[16] = the 32 values as 16 words, in
 // order) for the four MMA pairs of a quad lane: out[4w + 0..1] feed the first MMA of
 // packed word w, out[4w + 2..3] the second.
