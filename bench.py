@@ -499,7 +499,8 @@ def run_gpu(args):
     return 0
 
 
-CASES = ("quantize_70b", "gemv_m1_7b", "gemv_m4_7b", "gemv_m16_7b", "prefill", "prefill_w8")
+CASES = ("quantize_70b", "gemv_m1_7b", "gemv_m4_7b", "gemv_m16_7b", "gemv_m1_70b", "gemv_m8_70b",
+         "prefill", "prefill_w8")
 
 
 def run_case(name, reps):
@@ -526,7 +527,7 @@ def run_case(name, reps):
     elif name.startswith("gemv_m"):
         M = int(name[len("gemv_m"):].split("_")[0])
         work = []
-        for (N, K) in SHAPES:
+        for (N, K) in (wq_inputs.SHAPES_70B if name.endswith("_70b") else SHAPES):
             packed, S, Z = wq.wq_quantize_rtn_g128(bf16(wq_inputs.weight_bf16(N, K, 0.02)))
             work.append((bf16(wq_inputs.act_bf16(M, K)), packed, S, Z))
         for _ in range(reps):
