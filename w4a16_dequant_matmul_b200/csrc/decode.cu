@@ -260,9 +260,12 @@ gemv_decode(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restri
     }
     uint32_t frag[16];
     build_x_fragment(xw, frag);
+    // chunks of quarter c rotated by 2 (c >> 1): a warp's four quarter loads hit four bank groups
+    const int xrot = 2 * ((e >> 1) & 1);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      sts128(blk + 16 * j, make_uint4(frag[4 * j], frag[4 * j + 1], frag[4 * j + 2], frag[4 * j + 3]));
+      sts128(blk + 16 * ((j + xrot) & 3),
+             make_uint4(frag[4 * j], frag[4 * j + 1], frag[4 * j + 2], frag[4 * j + 3]));
     float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
     for (int v = 0; v < 16; ++v) ps[v & 3] += bf16_lo(xw[v]) + bf16_hi(xw[v]);
@@ -286,6 +289,8 @@ gemv_decode(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restri
   // stored, and the loads stay uniform
   const int xn = (lane >> 2) % M;  // token of this lane's fragment (duplicates past M)
   const uint32_t xf_lane = base_s + L.xf + xn * (G * 256) + c * 64;
+  // this lane's X fragment chunks 0, 1 sit at xlo, xlo + 16 and chunks 2, 3 at xhi, xhi + 16
+  const uint32_t xlo = 32u * (c >> 1), xhi = 32u - xlo;
   const uint32_t ring_lane = base_s + L.ring + r * pitch + 16 * c;
   uint32_t kMask = 0x00780078u, kMagic = 0x3F803F80u;  // register operands of the LOP3
   asm volatile("" : "+r"(kMask), "+r"(kMagic));
@@ -296,8 +301,8 @@ gemv_decode(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restri
                    float (&acc)[2][4]) {
     constexpr int RT = decltype(rt)::value;
     const uint32_t xs = xf_lane + g * 256;
-    const uint4 xb0 = lds128(xs), xb1 = lds128(xs + 16), xb2 = lds128(xs + 32),
-                xb3 = lds128(xs + 48);
+    const uint4 xb0 = lds128(xs + xlo), xb1 = lds128(xs + xlo + 16), xb2 = lds128(xs + xhi),
+                xb3 = lds128(xs + xhi + 16);
     const uint32_t bw[16] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w,
                              xb2.x, xb2.y, xb2.z, xb2.w, xb3.x, xb3.y, xb3.z, xb3.w};
     const float sx0 = sxs[g * 8 + t0];

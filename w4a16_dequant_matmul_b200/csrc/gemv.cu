@@ -577,9 +577,11 @@ gemv_mma_bulk(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __rest
     }
     uint32_t frag[16];
     build_x_fragment(xw, frag);
+    // chunks of quarter c rotated by 2 (c >> 1): a warp's four quarter loads hit four bank groups
     uint32_t* dst = xf + (static_cast<size_t>(g) * 4 * M + Lf) * 16;
+    const int xrot = 2 * ((Lf >> 1) & 1);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) dst[j] = frag[j];
+    for (int j = 0; j < 16; ++j) dst[(((j >> 2) + xrot) & 3) * 4 + (j & 3)] = frag[j];
   }
   for (int e = threadIdx.x; e < G * 8; e += 32 * NW) {
     const int g = e >> 3, n = e & 7;
@@ -604,6 +606,8 @@ gemv_mma_bulk(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __rest
   // lanes whose token column is >= M read a duplicate fragment: their columns are never
   // stored, and the loads stay uniform (no divergent branch)
   const uint32_t xf_lane = smem_u32(xf) + (lane % (4 * M)) * 64;
+  // this lane's X fragment chunks 0, 1 sit at xlo, xlo + 16 and chunks 2, 3 at xhi, xhi + 16
+  const uint32_t xlo = 32u * ((lane >> 1) & 1), xhi = 32u - xlo;
   const uint32_t ring_s = smem_u32(ring);
   const float* sx0p = sxs + t0;
   const float* sx1p = sxs + t1;
@@ -623,8 +627,8 @@ gemv_mma_bulk(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __rest
     for (int t = 0; t < RT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
     for (int g = g_lo; g < g_hi; ++g) {
       const uint32_t xs = xf_lane + g * (4 * M * 64);
-      const uint4 xb0 = lds128(xs), xb1 = lds128(xs + 16), xb2 = lds128(xs + 32),
-                  xb3 = lds128(xs + 48);
+      const uint4 xb0 = lds128(xs + xlo), xb1 = lds128(xs + xlo + 16), xb2 = lds128(xs + xhi),
+                  xb3 = lds128(xs + xhi + 16);
       const uint32_t bw[16] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w,
                                xb2.x, xb2.y, xb2.z, xb2.w, xb3.x, xb3.y, xb3.z, xb3.w};
       const float sx0 = sx0p[g * 8], sx1 = sx1p[g * 8];
