@@ -11,7 +11,7 @@
 // rows a quarter-warp reads sit 64 bytes apart and its 16-byte loads cover all 32 banks. The
 // tile's S' and Z (32 x G each, contiguous in HBM) arrive by two bulk copies into a slot of
 // their own. Before it waits for the previous kernel (programmatic dependent launch), each CTA
-// warms L2 with its first tiles (codes and S'/Z; hints only, so safe before the wait).
+// warms L2 with its codes past the first ring's worth (hints only, so safe before the wait).
 //
 // Warp roles:
 //   producer  one lane: X (one bulk copy per token), then per tile the S'/Z copies and the
@@ -114,14 +114,13 @@ gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X
   __syncthreads();
   if (threadIdx.x == 0) pdl_launch_dependents();
   if (warp == kNW && lane == 0) {
-    // warm L2 with this CTA's first tiles, codes and S'/Z (hints only): the reads then run
-    // at the full HBM rate, ahead of the ring
+    // warm L2 with this CTA's codes past the first NS chunks (hints only): those reads then
+    // run at the full HBM rate ahead of the ring, while the chunks the ring fetches at once
+    // keep the bandwidth to themselves (warming those too measured slower)
     prefetch_tensormap(&tmW);
-    for (int t = t_begin; t < t_end && t < t_begin + prefetch_tiles; ++t) {
-      prefetch_l2_bulk(S + static_cast<int64_t>(t) * kTR * G, szbytes);
-      prefetch_l2_bulk(Zp + static_cast<int64_t>(t) * kTR * G, szbytes);
-      for (int ch = 0; ch < NCH; ++ch) tma_prefetch_3d(&tmW, 0, t * kTR, ch * CG);
-    }
+    const int nchunks = (t_end - t_begin) * NCH;
+    for (int c = NS; c < nchunks && c < prefetch_tiles * NCH; ++c)
+      tma_prefetch_3d(&tmW, 0, (t_begin + c / NCH) * kTR, (c % NCH) * CG);
   }
   pdl_wait();
 
