@@ -464,11 +464,15 @@ def run_gpu(args):
                    "binding, Y D2H, stream sync; weights resident (quantized once)"}
 
     if rank == 0:
+        # DRAM traffic per step from the committed ncu capture, only while the decode kernels'
+        # sources are the ones it was taken with (else null)
         traffic = None
         tf = os.path.join(ROOT, "profiles", "gemv_traffic.json")
         if os.path.exists(tf):
             with open(tf) as f:
-                traffic = json.load(f).get("bytes_per_step")
+                rec = json.load(f)
+            if rec.get("sources_sha256") == decode_sources_sha256():
+                traffic = rec.get("bytes_per_step")
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -481,7 +485,8 @@ def run_gpu(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                         "peak_source": peak_src, "kernel": "gemv_mma_bulk (M=1)"},
+                         "peak_source": peak_src,
+                         "kernel": "gemv_mma_bulk (short rows) + gemv_tma (long rows), M=1"},
             "per_shape": per_shape,
             "secondary": secondary,
             "clocks": dict(clk.summary(), **({"soak_steps_after_timed_region": soak}
@@ -501,6 +506,20 @@ def run_gpu(args):
 
 CASES = ("quantize_70b", "gemv_m1_7b", "gemv_m4_7b", "gemv_m16_7b", "gemv_m1_70b", "gemv_m8_70b",
          "prefill", "prefill_w8")
+
+
+DECODE_SOURCES = ("gemv.cu", "gemv_tma.cu", "mma_frag.cuh", "ptx.cuh", "common.cuh", "kernels.h")
+
+
+def decode_sources_sha256():
+    """Hash of the sources the M = 1 decode kernels compile from (csrc/ of the package)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "w4a16_dequant_matmul_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def run_case(name, reps):
