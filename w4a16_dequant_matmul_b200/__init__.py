@@ -111,6 +111,28 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+_RAW_STREAM = None
+
+
+def _stream_handle(t, stream=None) -> int:
+    """cudaStream_t (as an int) of `stream`, or of the current stream of t's device; the
+    raw accessor avoids building a Stream object per call on the decode hot path."""
+    global _RAW_STREAM
+    if stream is not None:
+        return stream.cuda_stream
+    if _RAW_STREAM is None:
+        import torch
+
+        _RAW_STREAM = getattr(torch._C, "_cuda_getCurrentRawStream", None) or (
+            lambda dev: torch.cuda.current_stream(dev).cuda_stream)
+    dev = t.get_device()
+    if dev < 0:  # a host tensor: the library rejects it; any stream will do
+        import torch
+
+        dev = torch.cuda.current_device()
+    return _RAW_STREAM(dev)
+
+
 def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
@@ -233,17 +255,27 @@ def wq_dequant(packed, S, Z, group: int = 128, out_dtype=None, out=None, stream=
     return out
 
 
-def wq_w4a16_gemm(X, packed, S, Z, group: int = 128, Y=None, stream=None):
-    """Y [M, N] bf16 = X [M, K] bf16 @ W_hat^T, fp32 accumulation."""
-    import torch
+_GEMM = None
 
+
+def wq_w4a16_gemm(X, packed, S, Z, group: int = 128, Y=None, stream=None):
+    """Y [M, N] bf16 = X [M, K] bf16 @ W_hat^T, fp32 accumulation. (The decode hot path:
+    raw integer pointers and a cached function handle keep the per-call host cost low.)"""
+    global _GEMM
+    if _GEMM is None:
+        _GEMM = lib().wq_w4a16_gemm
     M, K = X.shape
     N = packed.shape[0]
     ldx = _rows(X, "X")
-    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device) if Y is None else Y
+    if Y is None:
+        import torch
+
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
     ldy = _rows(Y, "Y")
-    _check(lib().wq_w4a16_gemm(_ptr(X), M, ldx, _ptr(packed), _ptr(S), _ptr(Z), N, K, group,
-                               _ptr(Y), ldy, _stream(stream)), "wq_w4a16_gemm")
+    st = _GEMM(X.data_ptr(), M, ldx, packed.data_ptr(), S.data_ptr(), Z.data_ptr(), N, K, group,
+               Y.data_ptr(), ldy, _stream_handle(X, stream))
+    if st != 0:
+        raise WQError(st, "wq_w4a16_gemm")
     return Y
 
 
