@@ -356,13 +356,34 @@ cudaError_t launch_tma_m(const GemvArgs& a, int sms, cudaStream_t st) {
   if (ntiles == 0) return cudaSuccess;
   const TmaCfg c = tma_config(M, G);
   if (c.NS == 0) return cudaErrorInvalidValue;
-  CUtensorMap map;
-  // codes as [G groups][N rows][64 bytes]: boxes of CG groups x 32 rows x 64 bytes
-  const uint64_t dims[3] = {64, static_cast<uint64_t>(a.N), static_cast<uint64_t>(G)};
-  const uint64_t strides[2] = {static_cast<uint64_t>(a.K / 2), 64};
-  const uint32_t box[3] = {64, kTR, static_cast<uint32_t>(c.CG)};
-  if (!make_map_3d(&map, a.P, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8))
-    return cudaErrorInvalidValue;
+  // codes as [G groups][N rows][64 bytes]: boxes of CG groups x 32 rows x 64 bytes. The
+  // encoded map is kept per thread for the last few weight matrices (decode calls repeat).
+  struct MapEntry {
+    const void* p;
+    int n, k, cg;
+    CUtensorMap map;
+  };
+  constexpr int kMapCache = 16;
+  thread_local MapEntry cache[kMapCache];
+  thread_local int next_slot = 0;
+  const CUtensorMap* map = nullptr;
+  for (const MapEntry& e : cache)
+    if (e.p == a.P && e.n == a.N && e.k == a.K && e.cg == c.CG) map = &e.map;
+  if (!map) {
+    MapEntry& e = cache[next_slot];
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(a.N), static_cast<uint64_t>(G)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(a.K / 2), 64};
+    const uint32_t box[3] = {64, kTR, static_cast<uint32_t>(c.CG)};
+    e.p = nullptr;
+    if (!make_map_3d(&e.map, a.P, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+      return cudaErrorInvalidValue;
+    e.p = a.P;
+    e.n = a.N;
+    e.k = a.K;
+    e.cg = c.CG;
+    next_slot = (next_slot + 1) % kMapCache;
+    map = &e.map;
+  }
   const size_t smem = TmaLayout(M, G, c.NS, c.CG).total + kSlack;
   auto kern = gemv_tma<M>;
   static bool attr[64] = {false};
@@ -387,7 +408,7 @@ cudaError_t launch_tma_m(const GemvArgs& a, int sms, cudaStream_t st) {
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, map, a.X, a.ldx, a.S, a.Z, a.N, a.K, c.NS, c.CG,
+  return cudaLaunchKernelEx(&cfg, kern, *map, a.X, a.ldx, a.S, a.Z, a.N, a.K, c.NS, c.CG,
                             prefetch_tiles, a.Y, a.ldy, a.status);
 }
 
