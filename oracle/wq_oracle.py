@@ -50,6 +50,7 @@ __all__ = [
     "fp16_round", "bf16_round_bits", "bf16_bits_to_f64",
     "group_range", "asym_scale_zero", "quantize_rtn_asym", "pack_int4", "unpack_int4",
     "dequant_asym", "sym_scale", "quantize_sym_int8_per_channel", "dequant_sym_per_channel",
+    "Q4S_MIN", "Q4S_MAX", "quantize_rtn_sym_int4", "sym_int4_storage",
     "matmul_f64", "w4a16_matmul", "w8a16_matmul", "qdq_sym", "rel_frobenius",
     "gemm_gate", "bits_per_weight", "decode_ceiling_tok_s", "error_bound_ok",
     "outlier_quality",
@@ -57,6 +58,7 @@ __all__ = [
 
 Q4_MIN, Q4_MAX = 0, 15       # asymmetric INT4 integer range [CM]
 Q8_MAX = 127                  # symmetric INT8 integer range [CM]
+Q4S_MIN, Q4S_MAX = -8, 7      # symmetric INT4 range [-q_max - 1, q_max] [GR]
 FP16_MAX = 65504.0
 
 
@@ -231,6 +233,38 @@ def quantize_sym_int8_per_channel(W):
 
 def dequant_sym_per_channel(codes, s) -> np.ndarray:
     return np.asarray(codes, dtype=np.float64) * np.asarray(s, dtype=np.float64)[:, None]
+
+
+# ------------------------------------------------------ symmetric INT4 per group [GR]
+
+def quantize_rtn_sym_int4(W, group=128):
+    """Symmetric INT4 per group of g consecutive input weights [GR] ("quantize_per_group"):
+    s = max|w| / 7 over the group, stored as binary16 (RNE of the exact value; 0 -> 1.0),
+    q = clip(RNE(w/s'), -8, 7) on the exact quotient.
+
+    W: float array [N, K] of float32-representable values. Returns (q int8 [N, K],
+    S float64 [N, G] holding binary16 values)."""
+    W = np.asarray(W, dtype=np.float64)
+    if not np.all(np.isfinite(W)):
+        raise NonFiniteError("non-finite weight")
+    if not group:
+        raise ValueError("symmetric INT4 is defined per group here")
+    Wg = _groups(W, group)
+    R, G, _ = Wg.shape
+    S = np.empty((R, G))
+    for r in range(R):
+        for g in range(G):
+            S[r, g] = sym_scale(float(np.abs(Wg[r, g]).max()), Q4S_MAX)
+    # as in quantize_rtn_asym: rint of the float64 quotient is the RNE of the exact one
+    q = np.clip(np.rint(Wg / S[:, :, None]), Q4S_MIN, Q4S_MAX).astype(np.int8)
+    return q.reshape(W.shape), S
+
+
+def sym_int4_storage(q, S):
+    """The symmetric codes in the asymmetric INT4 storage (stored code q + 8, Z = 8), in
+    which S'(code - Z) = S' q: the format the library stores for zero_point = 0."""
+    codes = (np.asarray(q, dtype=np.int16) - Q4S_MIN).astype(np.uint8)
+    return codes, np.asarray(S, dtype=np.float64), np.full(np.shape(S), float(-Q4S_MIN))
 
 
 # -------------------------------------------------------------------- matmul [VO]

@@ -315,3 +315,82 @@ def test_outlier_quality_ordering():
     # output errors are reported, not ordered: with one outlier column they are dominated
     # by that column's rounding at any granularity
     assert all(0 < e[g][1] < 1 for g in e)
+
+
+# --------------------------------------------------- symmetric INT4 per group [GR]
+
+def _brute_sym_scale(w):
+    """s' by exhaustive nearest search over binary16 values of max|w| / 7 (ties to even)."""
+    allv = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    target = Fraction(float(np.abs(w).max())) / 7
+    j = bisect.bisect_left(allv.tolist(), float(target))
+    cands = [k for k in (j - 1, j, j + 1) if 0 <= k < len(allv)]
+    best = min(cands, key=lambda k: (abs(Fraction(float(allv[k])) - target), k % 2))
+    return float(allv[best]) or 1.0
+
+
+def _brute_sym_codes(w, s):
+    """Nearest of the 16 levels s*q, q in [-8, 7]; on a tie the even q."""
+    return [min(range(-8, 8), key=lambda q: (abs(Fraction(float(x)) - Fraction(s) * q), q % 2))
+            for x in w]
+
+
+def test_sym_int4_brute_force_tiny():
+    """Scale and codes against exhaustive searches: the nearest binary16 to max|w|/7, and
+    the nearest of the 16 levels s'q, ties to even q."""
+    rng = np.random.default_rng(21)
+    cases = [rng.normal(0, 0.02, 16), rng.normal(0.3, 0.01, 16), -np.abs(rng.normal(0, 1, 16)),
+             rng.normal(0, 1e-6, 16), rng.normal(0, 300.0, 16), np.zeros(16),
+             np.full(16, 0.37), np.full(16, -2.5)]
+    tie = np.array([0.5, -0.5, 1.5, -2.5, 3.5, 6.5, -6.5, 7.0]) * 0.25  # s' = 0.25 exactly
+    cases.append(tie)
+    for w in cases:
+        w = w.astype(np.float32).astype(np.float64)
+        q, S = oracle.quantize_rtn_sym_int4(w[None, :], len(w))
+        s_bf = _brute_sym_scale(w)
+        assert S[0, 0] == s_bf
+        assert q[0].tolist() == _brute_sym_codes(w, s_bf)
+
+
+def test_sym_int4_special_cases():
+    """All-zero group: s' = 1, q = 0. A constant group c maps to 7 (or -7): c/s' lies
+    within one binary16 step of 7. The ties of the exact grid go to even q."""
+    q, S = oracle.quantize_rtn_sym_int4(np.zeros((1, 32)), 32)
+    assert S[0, 0] == 1.0 and not q.any()
+    for c in (0.37, -2.5, 1e-3, 123.0):
+        q, _ = oracle.quantize_rtn_sym_int4(np.full((2, 64), c, dtype=np.float32).astype(np.float64), 32)
+        assert (q == (7 if c > 0 else -7)).all()
+    # group max 1.75 -> s' = 0.25 exactly; 0.125 * (2k + 1) are ties between k and k + 1
+    w = np.array([1.75] + [0.125 * (2 * k + 1) for k in range(-7, 7)] + [0.0])
+    q, S = oracle.quantize_rtn_sym_int4(w[None, :], len(w))
+    assert S[0, 0] == 0.25
+    expect = [7] + [k if k % 2 == 0 else k + 1 for k in range(-7, 7)] + [0]
+    assert q[0].tolist() == expect
+
+
+def test_sym_int4_equals_pinned_qdq_when_scale_exact():
+    """Where every group's max|w| / 7 is a binary16 value (so storing the scale changes
+    nothing), s'q equals qdq_sym(W, 4, group=g), which the printed granularity demo pins."""
+    rng = np.random.default_rng(22)
+    N, K, g = 8, 512, 128
+    W = rng.normal(0, 0.02, (N, K))
+    for r in range(N):
+        for j in range(K // g):
+            blk = W[r, j * g:(j + 1) * g]
+            m = float(np.float16(np.abs(blk).max() / 7)) * 7  # a group max that is 7 x binary16
+            blk *= m / np.abs(blk).max()
+    W = W.astype(np.float32).astype(np.float64)
+    q, S = oracle.quantize_rtn_sym_int4(W, g)
+    assert np.all(np.abs(W).reshape(N, -1, g).max(axis=-1) / 7 == S)  # scales exact
+    What = (q.reshape(N, -1, g) * S[:, :, None]).reshape(N, K)
+    assert np.array_equal(What, oracle.qdq_sym(W, 4, group=g))
+
+
+def test_sym_int4_storage_roundtrip():
+    """Stored as code q + 8 with Z = 8, the asymmetric dequant gives s'q exactly."""
+    W, _ = wq_inputs.tiny_config()
+    q, S = oracle.quantize_rtn_sym_int4(W.astype(np.float64), 128)
+    codes, S2, Z = oracle.sym_int4_storage(q, S)
+    assert codes.min() >= 0 and codes.max() <= 15 and (Z == 8).all()
+    assert np.array_equal(oracle.dequant_asym(codes, S2, Z, 128),
+                          (q.reshape(q.shape[0], -1, 128) * S[:, :, None]).reshape(q.shape))
