@@ -19,6 +19,9 @@
  *   - S' = binary16 round-half-even of the EXACT (beta - alpha)/15; S' = 0 -> 1.0;
  *   - Z = clip(round-half-even(-alpha/S'), 0, 15) on the exact quotient, stored binary16;
  *   - q = clip(round-half-even(w/S') + Z, 0, 15) on the exact quotient;
+ *   - INT4 symmetric per group ("DL S067 - Quantization", section 2, quantize_per_group):
+ *     s' = binary16(max|w|/7) (0 -> 1), q = clip(RNE(w/s'), -8, 7), stored in the INT4
+ *     layout below as code q + 8 with Z = 8, so dequant and matmul treat both alike;
  *   - INT8 symmetric: s' = binary16(max|w|/127), q = clip(RNE(w/s'), -127, 127).
  *
  * Data layout (row-major, all device memory owned by the caller):
@@ -68,12 +71,14 @@ typedef enum wq_status {
 typedef enum wq_dtype { WQ_F32 = 0, WQ_BF16 = 1, WQ_F16 = 2, WQ_U8 = 3, WQ_I8 = 4 } wq_dtype;
 
 /* Quantization parameters, named after the usual config keys (w_bit, q_group_size,
- * zero_point). Supported: {4, g, 1} with g a multiple of 32 that divides K (g = K is
- * per output channel), and {8, K, 0} (INT8 symmetric per channel). */
+ * zero_point). Supported: {4, g, 1} (asymmetric) and {4, g, 0} (symmetric, stored with
+ * Z = 8) with g a multiple of 32 that divides K (g = K is per output channel), and
+ * {8, K, 0} (INT8 symmetric per channel). */
 typedef struct wq_qparams {
   int32_t w_bit;      /* 4 or 8                                      */
   int32_t group;      /* g: weights per scale along K                 */
   int32_t zero_point; /* 1 = asymmetric [0, 15]; 0 = symmetric        */
+                      /*   (INT4: [-8, 7], stored as q + 8 with Z = 8) */
 } wq_qparams;
 
 /* Library version (WQ_VERSION) and a static description of a status code. */
@@ -84,7 +89,8 @@ const char* wq_status_string(wq_status status);
  *   W       fp32 or bf16 (w_dtype), row stride ldw >= K elements; base and row stride
  *           16-byte aligned.
  *   params  NULL means {4, 128, 1}.
- *   INT4 ({4, g, 1}): packed [N, K/2] uint8, S and Z [N, K/g] binary16.
+ *   INT4 ({4, g, 1} or {4, g, 0}): packed [N, K/2] uint8, S and Z [N, K/g] binary16
+ *           (symmetric: every Z is 8.0 and codes lie in [0, 15] as q + 8).
  *   INT8 ({8, K, 0}): packed receives int8 codes [N, K]; S [N] binary16; Z must be NULL.
  * Non-finite weights or a scale above the binary16 range set WQ_ERR_NONFINITE in the
  * device status word. Requires K % 32 == 0. */

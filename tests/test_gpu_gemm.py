@@ -209,3 +209,22 @@ def test_w8a16_small_m(M):
     Y = wq.wq_w8a16_gemm(gu.bf16_from_bits(Xb), q, S)
     Yref = oracle.w8a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), qo, so, "exact")
     assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 4096), (1, 64, 11008), (3, 160, 4096), (8, 128, 2048),
+                                   (64, 136, 1024)])
+def test_symmetric_int4_matmul(M, N, K):
+    """Symmetric INT4 weights (codes q + 8, Z = 8) through the same matmul kernels: the
+    decode kernels against the exact product, the tensor-core GEMM (M = 64) against the
+    bf16-rounded weights."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + K)
+    Xb = wq_inputs.act_bf16(M, K, seed=M + 9)
+    packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb), 4, 128, False)
+    q, So = oracle.quantize_rtn_sym_int4(wq_inputs.bf16_bits_to_f64(Wb), 128)
+    codes, So, Zo = oracle.sym_int4_storage(q, So)
+    np.testing.assert_array_equal(gu.to_np(packed), oracle.pack_int4(codes))
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    mode = "exact" if M <= 32 else "bf16"
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, mode)
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE

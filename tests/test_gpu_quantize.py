@@ -207,3 +207,73 @@ def test_empty_inputs():
                          torch.ones((5, 1), dtype=torch.float16, device="cuda"),
                          torch.zeros((5, 1), dtype=torch.float16, device="cuda"))
     assert Y.shape == (0, 5)
+
+
+# ------------------------------------------ symmetric INT4 per group (codes q + 8, Z = 8)
+
+def _check_sym4(W64, Wt, group):
+    packed, S, Z = wq.wq_quantize_rtn_g128(Wt, 4, group, False)
+    assert wq.wq_get_status() == 0
+    q, So = oracle.quantize_rtn_sym_int4(W64, group)
+    codes, So, Zo = oracle.sym_int4_storage(q, So)
+    np.testing.assert_array_equal(gu.bits16(S), gu.f16_bits_of(So))
+    np.testing.assert_array_equal(gu.bits16(Z), gu.f16_bits_of(Zo))
+    np.testing.assert_array_equal(gu.to_np(packed), oracle.pack_int4(codes))
+    return packed, S, Z, codes, So, Zo
+
+
+@pytest.mark.parametrize("group", [32, 128, 256, 384, 1152])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_sym4_random_shapes_and_groups(group, dtype):
+    N, K = 37, 1152
+    if dtype == "f32":
+        W = wq_inputs.to_f32(wq_inputs.normal_f64((N, K), 0.02, 4))
+        _check_sym4(W.astype(np.float64), gu.f32(W), group)
+    else:
+        Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=4)
+        _check_sym4(wq_inputs.bf16_bits_to_f64(Wb), gu.bf16_from_bits(Wb), group)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_sym4_adversarial_groups(dtype):
+    A = _adversarial_rows()
+    if dtype == "f32":
+        W = wq_inputs.to_f32(A)
+        _check_sym4(W.astype(np.float64), gu.f32(W), 128)
+    else:
+        Wb = wq_inputs.to_bf16_bits(A)
+        _check_sym4(wq_inputs.bf16_bits_to_f64(Wb), gu.bf16_from_bits(Wb), 128)
+
+
+def _sym_tie_lattice_bits():
+    """bf16 groups whose max|w| is 7 S0 with S0 = m 2^e a binary16 value, so s' = S0, holding
+    every exact tie (k + 1/2) S0 of the symmetric grid (k = -8..6) and fill; a second copy
+    moves half of the weights one bf16 ulp."""
+    rng = np.random.default_rng(98)
+    groups = []
+    for m in (1, 3, 5, 7, 9, 11, 13, 15, 17):
+        for e in (-20, -9, -3, 0, 5):
+            s0 = m * 2.0 ** e
+            for sign in (1.0, -1.0):
+                vals = [sign * 7 * s0] + [(k + 0.5) * s0 for k in range(-8, 7)]
+                g = np.resize(np.array(vals), 128)
+                g[len(vals):] = rng.uniform(-7 * s0, 7 * s0, 128 - len(vals))
+                groups.append(g)
+    bits = wq_inputs.to_bf16_bits(np.array(groups).reshape(-1, 256)).astype(np.int32)
+    move = (rng.random(bits.shape) < 0.5) & ((bits & 0x7FFF) != 0)
+    step = np.where(rng.random(bits.shape) < 0.5, 1, -1)
+    return np.concatenate([bits, np.where(move, bits + step, bits)]).astype(np.uint16)
+
+
+def test_sym4_tie_lattice_bf16():
+    Wb = _sym_tie_lattice_bits()
+    _check_sym4(wq_inputs.bf16_bits_to_f64(Wb), gu.bf16_from_bits(Wb), 128)
+
+
+def test_sym4_dequant_bitexact():
+    Wb = wq_inputs.weight_bf16(64, 1024, 0.02, seed=6)
+    packed, S, Z, codes, So, Zo = _check_sym4(wq_inputs.bf16_bits_to_f64(Wb),
+                                              gu.bf16_from_bits(Wb), 128)
+    W_hat = wq.wq_dequant(packed, S, Z, 128, torch.float32)
+    np.testing.assert_array_equal(gu.to_np(W_hat).astype(np.float64),
+                                  oracle.dequant_asym(codes, So, Zo, 128))

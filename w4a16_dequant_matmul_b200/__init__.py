@@ -164,7 +164,8 @@ def wq_status_string(status: int) -> str:
 def wq_quantize_rtn_g128(W, w_bit: int = 4, group: int = 128, zero_point: bool = True,
                          packed=None, S=None, Z=None, stream=None):
     """Round-to-nearest quantization of W [N, K]. INT4 asymmetric ({4, g, True}) returns
-    (packed uint8 [N, K/2], S fp16 [N, K/g], Z fp16 [N, K/g]); INT8 symmetric per channel
+    (packed uint8 [N, K/2], S fp16 [N, K/g], Z fp16 [N, K/g]); INT4 symmetric
+    ({4, g, False}) the same, with codes q + 8 and every Z = 8; INT8 symmetric per channel
     ({8, K, False}) returns (codes int8 [N, K], S fp16 [N], None)."""
     import torch
 

@@ -87,7 +87,7 @@ wq_status wq_quantize_rtn_g128(const void* W, wq_dtype w_dtype, int64_t N, int64
   const wq_qparams p = params ? *params : wq_qparams{4, 128, 1};
   if (N < 0 || K < 0) return WQ_ERR_SHAPE;
   if (w_dtype != WQ_F32 && w_dtype != WQ_BF16) return WQ_ERR_DTYPE;
-  const bool int4 = p.w_bit == 4 && p.zero_point == 1;
+  const bool int4 = p.w_bit == 4 && (p.zero_point == 1 || p.zero_point == 0);
   const bool int8 = p.w_bit == 8 && p.zero_point == 0;
   if (!int4 && !int8) return WQ_ERR_UNSUPPORTED;
   if (N == 0 || K == 0) return WQ_OK;
@@ -106,7 +106,7 @@ wq_status wq_quantize_rtn_g128(const void* W, wq_dtype w_dtype, int64_t N, int64
   const bool bf16 = w_dtype == WQ_BF16;
   if (int4)
     return from_cuda(wq::launch_quant_asym(W, bf16, ldw, (int)N, (int)K, p.group, packed, S, Z,
-                                           d->status, d->sms, st));
+                                           p.zero_point == 0, d->status, d->sms, st));
   return from_cuda(wq::launch_quant_sym_int8(W, bf16, ldw, (int)N, (int)K,
                                              reinterpret_cast<int8_t*>(packed), S, d->status,
                                              d->sms, st));

@@ -164,6 +164,16 @@ __device__ __forceinline__ AsymScale sym_scale(float amax, float qmax) {
   return r;
 }
 
+// Symmetric INT4 per group in the asymmetric storage ("DL S067 - Quantization", section 2,
+// quantize_per_group): s' = binary16 RNE(max|w| / 7) (0 -> 1) and Z = 8, so that the
+// asymmetric encode clip(RNE(w/s') + 8, 0, 15) stores clip(RNE(w/s'), -8, 7) + 8 and every
+// dequant s'(code - Z) is s'q. mn = min(0, min w), mx = max(0, max w) (NaN if a weight was).
+__device__ __forceinline__ AsymScale sym4_scale_zero(float mn, float mx) {
+  AsymScale r = sym_scale(fmax_nan(-mn, mx), 7.0f);
+  r.z = 8.0f;
+  return r;
+}
+
 // bf16 pair (one 32-bit word) -> two floats.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

@@ -11,9 +11,10 @@ namespace wq {
 // is no usable sm_100 device). Defined in api.cu.
 bool current_device(int* sms, unsigned** status);
 
+// sym: symmetric INT4 (s' = max|w|/7, Z = 8) in the same storage.
 cudaError_t launch_quant_asym(const void* W, bool bf16, int64_t ldw, int N, int K, int group,
-                              uint8_t* packed, uint16_t* S, uint16_t* Z, unsigned* status,
-                              int sms, cudaStream_t st);
+                              uint8_t* packed, uint16_t* S, uint16_t* Z, bool sym,
+                              unsigned* status, int sms, cudaStream_t st);
 cudaError_t launch_quant_sym_int8(const void* W, bool bf16, int64_t ldw, int N, int K,
                                   int8_t* codes, uint16_t* S, unsigned* status, int sms,
                                   cudaStream_t st);

@@ -186,7 +186,7 @@ template <typename T, int GS>
 __global__ void __launch_bounds__(128, 4)
 quant_asym_lanegroup(const T* __restrict__ W, int64_t ldw, int N, int K,
                      uint8_t* __restrict__ packed, uint16_t* __restrict__ S,
-                     uint16_t* __restrict__ Z, unsigned* status) {
+                     uint16_t* __restrict__ Z, bool sym, unsigned* status) {
   using Cfg = LaneGroupCfg<T, GS>;
   constexpr bool kBf16 = sizeof(T) == 2;
   constexpr int kChunks = Cfg::kChunks;
@@ -284,7 +284,7 @@ quant_asym_lanegroup(const T* __restrict__ W, int64_t ldw, int N, int K,
         }
       }
     }
-    const AsymScale sz = asym_scale_zero(mn, mx);
+    const AsymScale sz = sym ? sym4_scale_zero(mn, mx) : asym_scale_zero(mn, mx);
     // The snap path needs bf16 weights and a finite range (then |w/S'| < 32). Codes of the
     // range ends decide whether any code needs the clip; the whole warp then takes the
     // clipping variant, so that the warp does not split.
@@ -320,7 +320,7 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 quant_asym_wide(const T* __restrict__ W, int64_t ldw, int N, int K, int group,
                 uint8_t* __restrict__ packed, uint16_t* __restrict__ S,
-                uint16_t* __restrict__ Z, unsigned* status) {
+                uint16_t* __restrict__ Z, bool sym, unsigned* status) {
   const int G = K / group;
   const int64_t total = static_cast<int64_t>(N) * G;
   const int lane = threadIdx.x & 31;
@@ -341,7 +341,7 @@ quant_asym_wide(const T* __restrict__ W, int64_t ldw, int N, int K, int group,
       mn = fmin_nan(mn, __shfl_xor_sync(0xffffffffu, mn, o));
       mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    const AsymScale sz = asym_scale_zero(mn, mx);
+    const AsymScale sz = sym ? sym4_scale_zero(mn, mx) : asym_scale_zero(mn, mx);
     uint8_t* dst = packed + n * (K / 2) + static_cast<int64_t>(g) * (group / 2);
     for (int k = lane * 8; k < group; k += 256) {
       float v[8];
@@ -482,7 +482,8 @@ int grid_for(int64_t work_items, int per_block, int sms) {
 // blocks loop over the rest), so that no block starts after the others have finished.
 template <typename T, int GS>
 void launch_lanegroup(const T* W, int64_t ldw, int N, int K, uint8_t* packed, uint16_t* S,
-                      uint16_t* Z, unsigned* status, int64_t groups, int sms, cudaStream_t st) {
+                      uint16_t* Z, bool sym, unsigned* status, int64_t groups, int sms,
+                      cudaStream_t st) {
   using Cfg = LaneGroupCfg<T, GS>;
   static int per_sm = 0;  // resident blocks per SM (the same on every sm_100 device)
   if (per_sm == 0) {
@@ -498,20 +499,23 @@ void launch_lanegroup(const T* W, int64_t ldw, int N, int K, uint8_t* packed, ui
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   quant_asym_lanegroup<T, GS><<<static_cast<int>(blocks), 32 * Cfg::kWarps, 0, st>>>(
-      W, ldw, N, K, packed, S, Z, status);
+      W, ldw, N, K, packed, S, Z, sym, status);
 }
 
 template <typename T>
 cudaError_t launch_quant_asym_t(const T* W, int64_t ldw, int N, int K, int group,
-                                uint8_t* packed, uint16_t* S, uint16_t* Z, unsigned* status,
-                                int sms, cudaStream_t st) {
+                                uint8_t* packed, uint16_t* S, uint16_t* Z, bool sym,
+                                unsigned* status, int sms, cudaStream_t st) {
   const int64_t groups = static_cast<int64_t>(N) * (K / group);
   switch (group) {
-    case 32: launch_lanegroup<T, 32>(W, ldw, N, K, packed, S, Z, status, groups, sms, st); break;
-    case 64: launch_lanegroup<T, 64>(W, ldw, N, K, packed, S, Z, status, groups, sms, st); break;
-    case 128: launch_lanegroup<T, 128>(W, ldw, N, K, packed, S, Z, status, groups, sms, st); break;
-    case 256: launch_lanegroup<T, 256>(W, ldw, N, K, packed, S, Z, status, groups, sms, st); break;
-    default: quant_asym_wide<T><<<grid_for(groups, 8, sms), 256, 0, st>>>(W, ldw, N, K, group, packed, S, Z, status); break;
+    case 32: launch_lanegroup<T, 32>(W, ldw, N, K, packed, S, Z, sym, status, groups, sms, st); break;
+    case 64: launch_lanegroup<T, 64>(W, ldw, N, K, packed, S, Z, sym, status, groups, sms, st); break;
+    case 128: launch_lanegroup<T, 128>(W, ldw, N, K, packed, S, Z, sym, status, groups, sms, st); break;
+    case 256: launch_lanegroup<T, 256>(W, ldw, N, K, packed, S, Z, sym, status, groups, sms, st); break;
+    default:
+      quant_asym_wide<T><<<grid_for(groups, 8, sms), 256, 0, st>>>(W, ldw, N, K, group, packed,
+                                                                   S, Z, sym, status);
+      break;
   }
   return cudaGetLastError();
 }
@@ -519,12 +523,12 @@ cudaError_t launch_quant_asym_t(const T* W, int64_t ldw, int N, int K, int group
 }  // namespace
 
 cudaError_t launch_quant_asym(const void* W, bool bf16, int64_t ldw, int N, int K, int group,
-                              uint8_t* packed, uint16_t* S, uint16_t* Z, unsigned* status,
-                              int sms, cudaStream_t st) {
+                              uint8_t* packed, uint16_t* S, uint16_t* Z, bool sym,
+                              unsigned* status, int sms, cudaStream_t st) {
   if (bf16)
     return launch_quant_asym_t(static_cast<const uint16_t*>(W), ldw, N, K, group, packed, S, Z,
-                               status, sms, st);
-  return launch_quant_asym_t(static_cast<const float*>(W), ldw, N, K, group, packed, S, Z,
+                               sym, status, sms, st);
+  return launch_quant_asym_t(static_cast<const float*>(W), ldw, N, K, group, packed, S, Z, sym,
                              status, sms, st);
 }
 
