@@ -383,6 +383,33 @@ def run_gpu(args):
         else:
             secondary[f"gemv_M{M}_GB/s"] = round(tot_b / tot_us / 1e3, 1)
 
+    # ---- secondary: W8A16 decode (INT8 per-channel weights) at M = 1 on the same shapes,
+    # rotating weight sets larger than L2
+    try:
+        base8 = []
+        for (N, K) in SHAPES:
+            Wt = torch.from_numpy(wq_inputs.weight_bf16(N, K, 0.02).view(np.int16)).view(torch.bfloat16).to(dev)
+            q8, s8, _ = wq.wq_quantize_rtn_g128(Wt, 8, K, False)
+            base8.append((q8, s8))
+            del Wt
+        set8 = sum(q.numel() + 2 * s.numel() for q, s in base8)
+        n8 = max(2, math.ceil(3 * l2 / set8))
+        sets8 = [[(q.clone(), s.clone()) for q, s in base8] for _ in range(n8)]
+        tot_b, tot_us = 0, 0.0
+        for j, (N, K) in enumerate(SHAPES):
+            k = [0]
+
+            def one8(j=j, k=k):
+                q, s = sets8[k[0] % n8][j]
+                k[0] += 1
+                wq.wq_w8a16_gemm(X[j], q, s, Y=Y[j])
+            tot_us += graph_time_us(one8, 4 * n8)
+            tot_b += N * K + 2 * N + 2 * K + 2 * N  # codes, scales, x, y
+        secondary["w8a16_decode_M1_GB/s"] = round(tot_b / tot_us / 1e3, 1)
+        del sets8, base8
+    except wq.WQError as e:
+        secondary["w8a16_decode_M1_GB/s"] = f"unavailable: {e}"
+
     # ---- secondary: quantizer over the 70B-class weights, then the 70B decode layer
     # (M = 1, 8, 32) on the two quantized matrices, alternating (250 MB > L2)
     qres, q70 = {}, []
