@@ -9,11 +9,14 @@ Weights cycle through rotating copies totalling more than 3x the L2 cache, so ev
 launch streams its weights from HBM. Timing: CUDA graphs of the steps, CUDA events on the
 capturing stream, barrier + synchronize on both sides, max over ranks.
 
-Also reported (outside the timed step): M = 4, 8, 16 and 32 on the same shapes, the
-quantizer over the 70B-class weights (28672 x 8192, 8192 x 28672) and the 70B decode layer
-at M = 1, 8 and 32 on them, the prefill GEMM (2048 x 4096 x 11008) in W4A16 and in W8A16,
-the oracle on the host cores (cpu_baseline) and the end-to-end rate through host buffers
-(e2e).
+Also reported (outside the timed step): per-shape times of the step, M = 4, 8, 16 and 32
+on the same shapes, W8A16 decode at M = 1 on them, the quantizer over the 70B-class weights
+(28672 x 8192, 8192 x 28672) and the 70B decode layer at M = 1, 8 and 32 on them, the
+prefill GEMM (2048 x 4096 x 11008) in W4A16 and in W8A16, the oracle on the host cores
+(cpu_baseline) and the end-to-end rate through host buffers (e2e: one H2D copy of the
+step's X rows, the three calls, one D2H copy of its Y rows, a synchronize).
+roofline.traffic comes from profiles/gemv_traffic.json while the decode kernels' sources
+match the hash recorded there.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
