@@ -71,6 +71,10 @@ def test_quantize_argument_checks(lib):
     assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(3, 128), FAKE, FAKE, FAKE, None) == UNSUP
     assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(8, 128, 0), FAKE, FAKE, FAKE, None) == UNSUP
     assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(8, 64, 0), FAKE, FAKE, None, None) == UNSUP
+    # symmetric INT4 ({4, g, 0}) takes the INT4 checks: Z required, g a multiple of 32 dividing K
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(4, 128, 0), FAKE, FAKE, None, None) == NULL
+    assert f(FAKE, wq.WQ_BF16, 4, 192, 192, _qp(4, 128, 0), FAKE, FAKE, FAKE, None) == SHAPE
+    assert f(FAKE, wq.WQ_BF16, 4, 128, 128, _qp(4, 128, 2), FAKE, FAKE, FAKE, None) == UNSUP
     assert f(ODD, wq.WQ_BF16, 4, 128, 128, None, FAKE, FAKE, FAKE, None) == ALIGN
     assert f(FAKE, wq.WQ_BF16, 4, 128, 132, None, FAKE, FAKE, FAKE, None) == ALIGN   # row stride
     assert f(FAKE, wq.WQ_BF16, 4, 128, 128, None, ODD, FAKE, FAKE, None) == ALIGN
@@ -110,4 +114,7 @@ def test_valid_call_without_device_reports_nodevice(lib):
     """A call that passes every host check but finds no sm_100 device fails loudly
     (WQ_ERR_NODEVICE), and the Python binding raises: there is no CPU fallback."""
     assert lib.wq_w4a16_gemm(FAKE, 1, 128, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 64, None) == NODEV
+    sym = ctypes.byref(wq._QParams(4, 128, 0))
+    assert lib.wq_quantize_rtn_g128(FAKE, wq.WQ_BF16, 4, 128, 128, sym, FAKE, FAKE, FAKE,
+                                    None) == NODEV
     assert lib.wq_get_status(None) in (NODEV, 6)
