@@ -31,6 +31,8 @@ Readings where the pages are silent (each is pinned by a test in tests/test_orac
     S' is a binary16 subnormal far below S), stored as binary16;
   * codes use the exact quotient w/S', rounded half to even;
   * packed layout: row-major [N, K/2], byte j = q[2j] | q[2j+1] << 4;
+  * symmetric INT4 per group [GR]: s = max|w|/7 rounded once to binary16 (0 -> 1.0),
+    q = clip(RNE(w/s'), -8, 7) on the exact quotient, stored as q + 8 with Z = 8;
   * a matmul "on the same dequantized weights" uses either the exact S'(q - Z)
     ("exact" mode) or its bfloat16 rounding ("bf16" mode).
 
