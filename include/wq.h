@@ -174,6 +174,14 @@ wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t*
  * kernel since the last call; WQ_ERR_CUDA if the synchronization itself failed. */
 wq_status wq_get_status(void* stream);
 
+/* Self-test of failure detection: launches one CTA whose single mbarrier wait (on a barrier
+ * nothing arrives at) is bounded by limit_ns nanoseconds, with the same bounded wait the
+ * pipelined kernels use (spin != 0: the spinning form, else the suspending one). The wait
+ * gives up, records WQ_ERR_TIMEOUT in the device status word and the kernel returns; the
+ * next wq_get_status() reports it and clears it, and the context stays usable. No fault, trap
+ * or unbounded wait is involved. limit_ns in [1e3, 1e9], else WQ_ERR_SHAPE. */
+wq_status wq_selftest_bounded_wait(uint64_t limit_ns, int32_t spin, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -97,6 +97,12 @@ def test_gemm_argument_checks(lib):
     assert h(FAKE, 1, 128, FAKE, FAKE, 64, 100, FAKE, 64, None) == SHAPE
 
 
+def test_selftest_argument_checks(lib):
+    f = lib.wq_selftest_bounded_wait
+    assert f(0, 1, None) == SHAPE
+    assert f(2_000_000_000, 0, None) == SHAPE
+
+
 def test_pack_dequant_argument_checks(lib):
     assert lib.wq_pack_int4(FAKE, 4, 100, FAKE, None) == SHAPE
     assert lib.wq_pack_int4(None, 4, 128, FAKE, None) == NULL
@@ -114,6 +120,7 @@ def test_valid_call_without_device_reports_nodevice(lib):
     """A call that passes every host check but finds no sm_100 device fails loudly
     (WQ_ERR_NODEVICE), and the Python binding raises: there is no CPU fallback."""
     assert lib.wq_w4a16_gemm(FAKE, 1, 128, FAKE, FAKE, FAKE, 64, 128, 128, FAKE, 64, None) == NODEV
+    assert lib.wq_selftest_bounded_wait(20_000_000, 1, None) == NODEV
     sym = ctypes.byref(wq._QParams(4, 128, 0))
     assert lib.wq_quantize_rtn_g128(FAKE, wq.WQ_BF16, 4, 128, 128, sym, FAKE, FAKE, FAKE,
                                     None) == NODEV

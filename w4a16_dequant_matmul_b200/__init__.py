@@ -27,7 +27,7 @@ __all__ = [
     "wq_version", "wq_status_string", "wq_quantize_rtn_g128", "wq_quantize_rtn_per_tensor",
     "wq_quantize_per_tensor_workspace_bytes", "wq_quantize_rtn_per_tensor_noalloc",
     "wq_pack_int4", "wq_dequant", "wq_w4a16_gemm",
-    "wq_w8a16_gemm", "wq_get_status",
+    "wq_w8a16_gemm", "wq_get_status", "wq_selftest_bounded_wait",
     "WQ_F32", "WQ_BF16", "WQ_F16", "WQ_U8", "WQ_I8",
 ]
 
@@ -69,6 +69,7 @@ _SIGNATURES = {
     "wq_w4a16_gemm": (_I32, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I32, _P, _I64, _P]),
     "wq_w8a16_gemm": (_I32, [_P, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _P]),
     "wq_get_status": (_I32, [_P]),
+    "wq_selftest_bounded_wait": (_I32, [ctypes.c_uint64, _I32, _P]),
 }
 
 
@@ -292,6 +293,13 @@ def wq_w8a16_gemm(X, codes, S, Y=None, stream=None):
     _check(lib().wq_w8a16_gemm(_ptr(X), M, ldx, _ptr(codes), _ptr(S), N, K, _ptr(Y), ldy,
                                _stream(stream)), "wq_w8a16_gemm")
     return Y
+
+
+def wq_selftest_bounded_wait(limit_ns: int = 20_000_000, spin: bool = True, stream=None) -> None:
+    """Launch the failure-detection self-test (a bounded wait that runs out); the next
+    wq_get_status() then returns WQ_ERR_TIMEOUT (8)."""
+    _check(lib().wq_selftest_bounded_wait(int(limit_ns), 1 if spin else 0, _stream(stream)),
+           "wq_selftest_bounded_wait")
 
 
 def wq_get_status(stream=None) -> int:

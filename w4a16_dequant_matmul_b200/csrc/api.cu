@@ -246,6 +246,14 @@ wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t*
   return wq::launch_tc_gemm(a, d->sms, d->status, st);
 }
 
+wq_status wq_selftest_bounded_wait(uint64_t limit_ns, int32_t spin, void* stream) {
+  if (limit_ns < 1000u || limit_ns > 1000000000u) return WQ_ERR_SHAPE;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  return from_cuda(wq::launch_bounded_wait_selftest(limit_ns, spin != 0, d->status,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
 wq_status wq_get_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WQ_ERR_CUDA;
   const DeviceInfo* d = device_info();

@@ -65,4 +65,8 @@ struct Gemv8Args {
 };
 cudaError_t launch_gemv_w8a16(const Gemv8Args& a, cudaStream_t st);
 
+// One CTA whose single bounded mbarrier wait runs out (selftest.cu).
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, bool spin, unsigned* status,
+                                         cudaStream_t st);
+
 }  // namespace wq
