@@ -546,7 +546,7 @@ CASES = ("quantize_70b", "gemv_m1_7b", "gemv_m4_7b", "gemv_m16_7b", "gemv_m1_70b
          "prefill", "prefill_w8")
 
 
-DECODE_SOURCES = ("gemv.cu", "gemv_tma.cu", "mma_frag.cuh", "ptx.cuh", "common.cuh", "kernels.h")
+DECODE_SOURCES = ("gemv.cu", "gemv_tma.cu", "mma_frag.cuh", "ptx.cuh", "common.cuh")
 
 
 def decode_sources_sha256():
