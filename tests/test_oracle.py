@@ -394,3 +394,16 @@ def test_sym_int4_storage_roundtrip():
     assert codes.min() >= 0 and codes.max() <= 15 and (Z == 8).all()
     assert np.array_equal(oracle.dequant_asym(codes, S2, Z, 128),
                           (q.reshape(q.shape[0], -1, 128) * S[:, :, None]).reshape(q.shape))
+
+
+def test_sym_int4_hand_examples(golden_dir):
+    """Hand-worked symmetric INT4 groups (g = 4 on a 3 x 8 matrix, so a transposed grouping
+    fails): s', codes, the stored form (q + 8, Z = 8) and its packing."""
+    g = _load(golden_dir, "sym_int4_hand.json")
+    W = np.array(g["W"], dtype=np.float64)
+    q, S = oracle.quantize_rtn_sym_int4(W, g["group"])
+    assert S.tolist() == g["S"]
+    assert q.tolist() == g["q"]
+    codes, _, Z = oracle.sym_int4_storage(q, S)
+    assert (Z == 8).all()
+    assert oracle.pack_int4(codes)[0].tolist() == g["packed_row0"]
