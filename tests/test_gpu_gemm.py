@@ -149,9 +149,9 @@ def test_stream_many_tiles_sampled(N, K, M):
                                  (300, 8192), (48, 28672), (32, 40960)])
 def test_m1_decode_shapes(N, K):
     """M = 1 at assorted sizes: one row block, ragged row blocks, a row count just past a
-    multiple of the tile, K up to 11008, and K whose rows do not fit in shared memory whole
-    (28672, the 70B down projection, and 40960, past the register-loaded kernels): those
-    run on the streaming kernel in K chunks; bitwise repeatable."""
+    multiple of the tile, K up to 11008, and K whose rows do not fit in shared memory whole:
+    28672 (the 70B down projection's K) with N = 48 on the register-fed MMA kernel, and
+    40960 with N = 32 on the TMA-fed kernel in chunks of 8 groups; bitwise repeatable."""
     Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + 5 * K)
     Xb = wq_inputs.act_bf16(1, K, seed=K)
     packed, S, Z, codes, So, Zo = _quantize_both(Wb, 128)
