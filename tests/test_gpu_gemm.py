@@ -105,7 +105,9 @@ def test_full_size_decode_sampled(N, K):
     assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref) <= GATE
 
 
-# N a multiple of 16: the streaming decode kernel (16-row tiles, chunks of 4 groups)
+# N a multiple of 16, short and long rows: for M = 2..4 the streaming kernel on 16-row tiles
+# (short rows) and the TMA-fed kernel on 32-row tiles (K = 11008), for M = 1 the bulk-copy
+# kernel (short rows) and the TMA-fed one (K = 11008)
 STREAM_SHAPES = [(16, 128), (48, 384), (160, 1152), (32, 11008), (256, 4096)]
 
 
