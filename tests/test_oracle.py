@@ -407,3 +407,111 @@ def test_sym_int4_hand_examples(golden_dir):
     codes, _, Z = oracle.sym_int4_storage(q, S)
     assert (Z == 8).all()
     assert oracle.pack_int4(codes)[0].tolist() == g["packed_row0"]
+
+
+# ------------------------------------------- pins of the remaining checker functions
+
+def test_w8a16_matmul_modes():
+    """W8A16 on the same dequantized weights: exact mode = X (s' q)^T, bf16 mode rounds each
+    s' q to bfloat16 first; both against a per-element math.fsum loop, the bf16 weights
+    through torch's float32 -> bfloat16 cast (not the oracle's own rounding)."""
+    import torch
+    rng = np.random.default_rng(31)
+    W = rng.normal(0, 0.02, (5, 96)).astype(np.float32).astype(np.float64)
+    X = rng.normal(0, 1, (3, 96))
+    q, s = oracle.quantize_sym_int8_per_channel(W)
+    Y = oracle.w8a16_matmul(X, q, s, "exact")
+    Yb = oracle.w8a16_matmul(X, q, s, "bf16")
+    assert Y.shape == Yb.shape == (3, 5)
+    for n in range(5):
+        wh = [float(s[n]) * int(q[n, k]) for k in range(96)]
+        whb = torch.tensor(wh, dtype=torch.float32).to(torch.bfloat16).to(torch.float64).tolist()
+        # the bf16 rounding really moves some weights here, so the two modes differ
+        assert any(a != b for a, b in zip(wh, whb))
+        for m in range(3):
+            assert abs(Y[m, n] - math.fsum(X[m, k] * wh[k] for k in range(96))) < 1e-12
+            assert abs(Yb[m, n] - math.fsum(X[m, k] * whb[k] for k in range(96))) < 1e-12
+    with pytest.raises(ValueError):
+        oracle.w8a16_matmul(X, q, s, "fp8")
+
+
+def test_error_bound_ok_rejects_violations():
+    """error_bound_ok is a checker, so it must also say no: a dequantized weight moved to
+    just beyond S'/2 (+ 15 max(0, S - S')) from w is rejected, one exactly on the bound is
+    accepted. Two groups: one where binary16 rounded S up (bound S'/2) and one where it
+    rounded S down (bound widened by 15 (S - S'))."""
+    # group A: range 4.5 -> S = 0.3, S' = fp16(0.3) = 0.300048828125 > S
+    # group B: range 1.5 -> S = 0.1, S' = fp16(0.1) = 0.0999755859375 < S
+    wa = np.array([0.0, 4.5, 1.3, 2.2])
+    wb = np.array([0.0, 1.5, 0.7, 0.2])
+    W = np.stack([np.concatenate([wa, wb])]).astype(np.float32).astype(np.float64)
+    S = np.array([[0.300048828125, 0.0999755859375]])
+    assert S.tolist() == [[float(np.float16(0.3)), float(np.float16(0.1))]]
+    s_exact = [Fraction(9, 2) / 15, Fraction(3, 2) / 15]
+    assert Fraction(S[0, 0]) > s_exact[0] and Fraction(S[0, 1]) < s_exact[1]
+    bounds = [Fraction(S[0, 0]) / 2,
+              Fraction(S[0, 1]) / 2 + 15 * (s_exact[1] - Fraction(S[0, 1]))]
+    for g, elem in ((0, 2), (1, 6)):
+        for sign in (1, -1):
+            on = W.copy()
+            on[0, elem] = float(Fraction(float(W[0, elem])) + sign * bounds[g])
+            # the sum is exact in float64 here (a few bits each), so `on` sits on the bound
+            assert Fraction(on[0, elem]) - Fraction(float(W[0, elem])) == sign * bounds[g]
+            assert oracle.error_bound_ok(W, on, S, 4)
+            off = on.copy()
+            off[0, elem] = float(np.nextafter(on[0, elem], sign * np.inf))
+            assert not oracle.error_bound_ok(W, off, S, 4)
+    # an all-zero group has bound 0: any nonzero W_hat there is rejected
+    Wz = np.zeros((1, 4))
+    assert oracle.error_bound_ok(Wz, Wz, np.ones((1, 1)), 4)
+    assert not oracle.error_bound_ok(Wz, Wz + [[0, 0, 2.0 ** -30, 0]], np.ones((1, 1)), 4)
+
+
+def _brute_group_dequant(w):
+    """One group's dequantized weights from the brute-force searches alone: S' as the
+    nearest binary16 to the exact range / 15, Z and codes as the nearest levels."""
+    a, b = min(0.0, float(np.min(w))), max(0.0, float(np.max(w)))
+    s, z = _brute_scale(a, b)
+    return [s * (q - int(z)) for q in _brute_codes(w, s, z)]
+
+
+def _fsum_frobenius_rel(A, B):
+    """||A - B||_F / ||A||_F with exactly rounded sums of squares."""
+    num = math.fsum((float(x) - float(y)) ** 2 for x, y in zip(np.ravel(A), np.ravel(B)))
+    den = math.fsum(float(x) ** 2 for x in np.ravel(A))
+    return math.sqrt(num / den)
+
+
+def test_outlier_quality_brute_force():
+    """outlier_quality recomputed on a tiny outlier case (4 x 256, two outlier input
+    columns x 20-100, as "DL S067 - Quantization", "The origin story") from the brute-force
+    searches and fsum norms, at g = 128, per channel (g = K) and per tensor: both the
+    weight and the output error, so a wrong group axis, a per-tensor reshape bug or a
+    transposed product fails."""
+    rng = np.random.default_rng(41)
+    N, K, M = 4, 256, 3
+    W = rng.normal(0, 0.02, (N, K))
+    X = rng.normal(0, 1, (M, K))
+    cols = [17, 200]
+    W[:, cols] *= [37.0, 81.0]
+    X[:, cols] *= [55.0, 23.0]
+    W = W.astype(np.float32).astype(np.float64)
+    Y = [[math.fsum(X[m, k] * W[n, k] for k in range(K)) for n in range(N)] for m in range(M)]
+    results = {}
+    for group in (128, K, 0):
+        if group == 0:
+            flat = _brute_group_dequant(W.ravel())
+            What = np.array(flat).reshape(N, K)
+        else:
+            What = np.array([sum((_brute_group_dequant(W[n, j:j + group])
+                                  for j in range(0, K, group)), []) for n in range(N)])
+        Yq = [[math.fsum(X[m, k] * What[n, k] for k in range(K)) for n in range(N)]
+              for m in range(M)]
+        ref = (_fsum_frobenius_rel(W, What), _fsum_frobenius_rel(Y, Yq))
+        got = oracle.outlier_quality(W, X, group)
+        assert got[0] == pytest.approx(ref[0], rel=1e-12), group
+        assert got[1] == pytest.approx(ref[1], rel=1e-12), group
+        results[group] = got
+    # the three granularities really differ on this case
+    assert results[128][0] < results[K][0] < results[0][0]
+    assert len({round(v[1], 9) for v in results.values()}) == 3
