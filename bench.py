@@ -206,9 +206,37 @@ def cpu_baseline(target_s=10.0, rows=1024):
         tt += og.run()
         passes += 1
     return {"value": round(og.bytes * passes / tt / 1e9, 4), "unit": UNIT,
-            "cores": blas_threads(), "kind": "oracle",
+            "cores": blas_threads(), "host_cores": os.cpu_count(), "kind": "oracle",
+            "threading": "unpack and dequantize run single-threaded in numpy; only the fp64 "
+                         "matmul uses the BLAS threads counted in 'cores'",
             "sample": f"{rows} rows of each of the 3 shapes at M=1 (unpack + dequant + fp64 "
                       f"matmul), {passes} passes in {tt:.1f} s"}
+
+
+def c3_oracle_parity(Wb, gpu):
+    """The GPU quantizer's codes, S' and Z on the C3 outlier weights against the oracle: every
+    row at per tensor, 256 sampled rows (the first and last among them) at g = 128 and per
+    channel. Returns {granularity: bool}."""
+    import oracle
+
+    W = wq_inputs.bf16_bits_to_f64(Wb)
+    N = W.shape[0]
+    rows = np.sort(np.random.default_rng(3).choice(N, 256, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    out = {}
+    for name, (group, packed, S, Z) in gpu.items():
+        if group == 0:
+            codes, So, Zo = oracle.quantize_rtn_asym(W, 0)
+            ok = np.array_equal(packed, oracle.pack_int4(codes))
+        else:
+            codes, So, Zo = oracle.quantize_rtn_asym(W[rows], group)
+            ok = np.array_equal(packed[rows], oracle.pack_int4(codes))
+            S, Z = S[rows], Z[rows]
+        f16 = lambda v: np.asarray(v, dtype=np.float64).astype(np.float16).view(np.uint16)
+        ok = ok and np.array_equal(S.ravel(), f16(So).ravel()) and \
+            np.array_equal(Z.ravel(), f16(Zo).ravel())
+        out[name] = bool(ok)
+    return out
 
 
 def run_reference(args):
@@ -229,7 +257,8 @@ def run_reference(args):
         "data": "synthetic",
         "config": {"workload": WORKLOAD + f" (CPU oracle, {rows} sampled rows per shape per step)"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": blas_threads(),
-                         "kind": "oracle", "sample": f"{rows} rows of each of the 3 shapes per step"},
+                         "host_cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"{rows} rows of each of the 3 shapes per step"},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -300,7 +329,10 @@ def run_gpu(args):
         for j, (p, s, z) in enumerate(sets[i % nsets]):
             wq.wq_w4a16_gemm(X[j], p, s, z, 128, Y=Y[j])
 
-    # one graph per rotating set (a step each) and one graph of all sets (nsets steps)
+    # The timed steps run from CUDA graphs captured for exactly that count: one graph of all
+    # of them up to kMaxGraphSteps, else graphs of B steps (a multiple of the weight sets)
+    # and one of the remainder, so the timed region does not depend on how the step count
+    # divides into graphs (each graph boundary breaks the launch overlap between kernels).
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -308,42 +340,47 @@ def run_gpu(args):
             step(i)
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
-    g_one = []
-    for i in range(nsets):
+
+    def capture(nsteps):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step(i)
-        g_one.append(g)
-    g_all = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_all):
-        for i in range(nsets):
-            step(i)
+            for i in range(nsteps):
+                step(i)
+        return g
 
-    def run_steps(k, start=0):
-        i = start
-        while k - (i - start) >= nsets and (i % nsets) == 0:
-            g_all.replay()
-            i += nsets
-        while i - start < k:
-            g_one[i % nsets].replay()
-            i += 1
+    kMaxGraphSteps = 1024
+    if args.steps <= kMaxGraphSteps:
+        plan = [(capture(args.steps), 1)]
+    else:
+        B = nsets * math.ceil(512 / nsets)
+        plan = [(capture(B), args.steps // B)]
+        if args.steps % B:
+            plan.append((capture(args.steps % B), 1))
+    g_warm = capture(max(args.warmup, 3))
 
-    run_steps(max(args.warmup, 3))
+    def run_timed():
+        for g, reps in plan:
+            for _ in range(reps):
+                g.replay()
+
+    g_warm.replay()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
         barrier(world)
         torch.cuda.synchronize()
         ev0.record()
-        run_steps(args.steps)
+        run_timed()
         ev1.record()
         torch.cuda.synchronize()
         barrier(world)
         dt_local = ev0.elapsed_time(ev1) * 1e-3
         soak = 0
         if dt_local < 1.5 and not args.no_soak:  # keep the step graphs running for the sampler
-            soak = int(args.steps * 1.5 / max(dt_local, 1e-6))
-            run_steps(soak)
+            reps = int(1.5 / max(dt_local, 1e-6)) + 1
+            for _ in range(reps):
+                run_timed()
+            soak = reps * args.steps
             torch.cuda.synchronize()
     dt = ev0.elapsed_time(ev1) * 1e-3
     dt = max_over_ranks(dt, world)
@@ -444,6 +481,36 @@ def run_gpu(args):
     del q70
     assert wq.wq_get_status() == 0
 
+    # ---- secondary: outlier stress (C3): W 4096 x 4096 ~N(0, 0.02) with 0.1% of the input
+    # columns x U(20, 100), X 8 x 4096 with the same channels scaled; relative Frobenius errors
+    # of the weights and of Y = X W^T after GPU quantization at g = 128, per output channel
+    # (g = K) and per tensor. The codes are compared with the oracle in the CPU leg.
+    c3, c3_codes = {}, {}
+    Wb3, Xb3, cols3 = wq_inputs.outlier_config(N=4096, K=4096, M=8)
+    W3 = torch.from_numpy(Wb3.view(np.int16)).view(torch.bfloat16).to(dev)
+    X3 = torch.from_numpy(Xb3.view(np.int16)).view(torch.bfloat16).to(dev)
+    W3d, X3d = W3.double(), X3.double()
+    Y3ref = X3d @ W3d.T
+    for name, group in (("g128", 128), ("per_channel", 4096), ("per_tensor", 0)):
+        if group:
+            pk3, s3, z3 = wq.wq_quantize_rtn_g128(W3, 4, group, True)
+        else:
+            pk3, s3, z3 = wq.wq_quantize_rtn_per_tensor(W3)
+        What3 = wq.wq_dequant(pk3, s3, z3, group, torch.float32).double()
+        Y3 = wq.wq_w4a16_gemm(X3, pk3, s3, z3, group).double()
+        c3[name] = {
+            "weight_rel_err": round(float((W3d - What3).norm() / W3d.norm()), 6),
+            "output_rel_err": round(float((Y3ref - Y3).norm() / Y3ref.norm()), 6)}
+        c3_codes[name] = (group, pk3.cpu().numpy(), s3.cpu().numpy().view(np.uint16),
+                          z3.cpu().numpy().view(np.uint16))
+    assert wq.wq_get_status() == 0
+    c3["weight_err_order_g128_lt_channel_lt_tensor"] = bool(
+        c3["g128"]["weight_rel_err"] < c3["per_channel"]["weight_rel_err"]
+        < c3["per_tensor"]["weight_rel_err"])
+    c3["outlier_columns"] = [int(c) for c in cols3]
+    secondary["c3_outlier"] = c3
+    del W3, X3, W3d, X3d, Y3ref
+
     # ---- secondary: prefill GEMM (tensor cores)
     prefill = None
     try:
@@ -524,7 +591,8 @@ def run_gpu(args):
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                          "peak_source": peak_src,
-                         "kernel": "gemv_mma_bulk (short rows) + gemv_tma (long rows), M=1"},
+                         "kernel": "gemv_imma_bulk (4096x4096, 11008x4096) + gemv_tma "
+                                   "integer path (4096x11008), M=1"},
             "per_shape": per_shape,
             "secondary": secondary,
             "clocks": dict(clk.summary(), **({"soak_steps_after_timed_region": soak}
@@ -533,8 +601,10 @@ def run_gpu(args):
             "gpu_launches": len(SHAPES) * args.steps,
             "cpu_baseline": cpu_baseline() if not args.no_cpu_baseline else None,
         }
+        if not args.no_cpu_baseline:
+            secondary["c3_outlier"]["bitexact_vs_oracle"] = c3_oracle_parity(Wb3, c3_codes)
         print(json.dumps(line), flush=True)
-    del g_one, g_all
+    del plan, g_warm
     if world > 1:
         import torch.distributed as dist
 
@@ -546,7 +616,8 @@ CASES = ("quantize_70b", "gemv_m1_7b", "gemv_m4_7b", "gemv_m16_7b", "gemv_m1_70b
          "prefill", "prefill_w8")
 
 
-DECODE_SOURCES = ("gemv.cu", "gemv_tma.cu", "mma_frag.cuh", "ptx.cuh", "common.cuh")
+DECODE_SOURCES = ("gemv.cu", "gemv_imma.cu", "gemv_tma.cu", "imma_digits.cuh", "mma_frag.cuh",
+                  "ptx.cuh", "common.cuh")
 
 
 def decode_sources_sha256():

@@ -31,9 +31,11 @@
  *   X      [M, K] bf16, leading dimension ldx; Y [M, N] bf16, leading dimension ldy
  *
  * Conventions:
- *   - Every pointer argument is a DEVICE pointer owned by the caller, unless stated.
- *     The library allocates no device memory; a small device status word and the
- *     kernels' code are module globals.
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless stated, in
+ *     memory of the CURRENT device (cudaSetDevice) or managed memory; any other pointer
+ *     (host memory, pinned or not, or another device's memory) is rejected with
+ *     WQ_ERR_DEVICE before anything is launched. The library allocates no device memory;
+ *     a small device status word and the kernels' code are module globals.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
  *     legacy default stream) on the current device.
  *   - Argument errors are returned synchronously and launch nothing. A failed launch
@@ -65,7 +67,8 @@ typedef enum wq_status {
   WQ_ERR_NONFINITE = 7,   /* device: NaN/inf weight or binary16 scale overflow   */
   WQ_ERR_TIMEOUT = 8,     /* device: a bounded barrier wait gave up              */
   WQ_ERR_RANGE = 9,       /* device: a code given to wq_pack_int4 exceeds 15     */
-  WQ_ERR_NODEVICE = 10    /* no CUDA device, or it is not sm_100                 */
+  WQ_ERR_NODEVICE = 10,   /* no CUDA device, or it is not sm_100                 */
+  WQ_ERR_DEVICE = 11      /* a pointer is not memory of the current device      */
 } wq_status;
 
 typedef enum wq_dtype { WQ_F32 = 0, WQ_BF16 = 1, WQ_F16 = 2, WQ_U8 = 3, WQ_I8 = 4 } wq_dtype;

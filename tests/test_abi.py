@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     assert wq.wq_version() == 100
-    for code in range(11):
+    for code in range(12):
         s = wq.wq_status_string(code)
         assert s and s != "unknown status"
     assert wq.wq_status_string(99) == "unknown status"
@@ -125,3 +125,69 @@ def test_valid_call_without_device_reports_nodevice(lib):
     assert lib.wq_quantize_rtn_g128(FAKE, wq.WQ_BF16, 4, 128, 128, sym, FAKE, FAKE, FAKE,
                                     None) == NODEV
     assert lib.wq_get_status(None) in (NODEV, 6)
+
+
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor on device `dev` (nothing is ever dereferenced)."""
+
+    def __init__(self, shape, dev, addr=0x10000):
+        self.shape = shape
+        self._dev = dev
+        self._addr = addr
+
+    def get_device(self):
+        return self._dev
+
+    def dim(self):
+        return len(self.shape)
+
+    def stride(self, i=None):
+        st = (self.shape[1], 1)
+        return st if i is None else st[i]
+
+    def data_ptr(self):
+        return self._addr
+
+
+def test_binding_makes_the_tensors_device_current(monkeypatch):
+    """The C library works on the current device and rejects other devices' memory, so the
+    binding switches to the device that holds the tensors for the call (host-side mock: a
+    tensor "on cuda:1" while cuda:0 is current; no GPU is touched)."""
+    import torch
+
+    current = [0]
+    seen = []
+
+    class _Dev:
+        def __init__(self, d):
+            self.d = d
+
+        def __enter__(self):
+            self.prev, current[0] = current[0], self.d
+
+        def __exit__(self, *exc):
+            current[0] = self.prev
+
+    monkeypatch.setattr(torch.cuda, "device", _Dev)
+    monkeypatch.setattr(wq, "_GET_DEVICE", lambda: current[0])
+
+    def fake_gemm(*args):
+        seen.append(current[0])
+        return 0
+
+    monkeypatch.setattr(wq, "_GEMM", fake_gemm)
+
+    class _Stream:
+        cuda_stream = 0
+
+    M, N, K = 1, 64, 128
+    X = _FakeCudaTensor((M, K), 1)
+    P = _FakeCudaTensor((N, K // 2), 1)
+    S = _FakeCudaTensor((N, 1), 1)
+    Y = _FakeCudaTensor((M, N), 1)
+    wq.wq_w4a16_gemm(X, P, S, S, 128, Y=Y, stream=_Stream())
+    assert seen == [1] and current[0] == 0, "called on the tensors' device, then restored"
+    # tensors already on the current device: no switch
+    X0, P0, S0, Y0 = (_FakeCudaTensor(t.shape, 0) for t in (X, P, S, Y))
+    wq.wq_w4a16_gemm(X0, P0, S0, S0, 128, Y=Y0, stream=_Stream())
+    assert seen == [1, 0]

@@ -230,3 +230,96 @@ def test_symmetric_int4_matmul(M, N, K):
     mode = "exact" if M <= 32 else "bf16"
     Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, mode)
     assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE
+
+
+def test_host_memory_is_rejected_before_launch():
+    """Pointers that are not memory of the current device are refused with WQ_ERR_DEVICE
+    before anything is launched (pinned host memory here: even a launch would only have
+    read it through unified addressing, so the check itself is what the test observes)."""
+    N, K = 64, 1024
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=5)
+    packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb))
+    Xh = torch.zeros((1, K), dtype=torch.bfloat16).pin_memory()
+    Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_w4a16_gemm(Xh, packed, S, Z, 128, Y=Y)
+    assert e.value.status == 11
+    Ph = packed.cpu().pin_memory()
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_dequant(Ph, S, Z, 128)
+    assert e.value.status == 11
+    assert wq.wq_get_status() == 0
+
+
+def _sampled_rows(N, k, seed):
+    rows = np.sort(np.random.default_rng(seed).choice(N, k, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    return rows
+
+
+@pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672)])
+@pytest.mark.parametrize("M", [8, 32])
+def test_70b_skinny_sampled(N, K, M):
+    """70B-class decode layers at M = 8 and 32 in the benchmark's configuration (the whole W
+    quantized and multiplied on the GPU); the oracle quantizes and multiplies 64 sampled rows,
+    the first and last among them. M = 8 runs as token blocks on the decode kernels (exact
+    S'(q - Z)); M = 32 at K = 28672 needs more than 8 blocks there and runs on the tensor-core
+    GEMM, which rounds S'(q - Z) to bf16 first, so it is compared with that mode."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.015)
+    Xb = wq_inputs.act_bf16(M, K)
+    packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb))
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    rows = _sampled_rows(N, 64, N + M)
+    codes, So, Zo = oracle.quantize_rtn_asym(wq_inputs.bf16_bits_to_f64(Wb[rows]), 128)
+    np.testing.assert_array_equal(gu.to_np(packed)[rows], oracle.pack_int4(codes))
+    mode = "bf16" if (M == 32 and K == 28672) else "exact"
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, mode)
+    y = gu.bf16_to_f64(Y)[:, rows]
+    assert oracle.gemm_gate(y, Yref) <= GATE
+    assert oracle.rel_frobenius(Yref, y) < 4e-3
+
+
+@pytest.mark.parametrize("group", [4096, 0])
+def test_outlier_config_m8_channel_and_tensor(group):
+    """The outlier-stress configuration itself (W 4096 x 4096 with 0.1% of the input columns
+    scaled x20-100, X 8 x 4096 with the same channels scaled) at per-channel and per-tensor
+    scales: codes, S' and Z bit-exact against the oracle (all rows per tensor, sampled rows
+    per channel), and Y on sampled rows within the gate."""
+    Wb, Xb, _ = wq_inputs.outlier_config(N=4096, K=4096, M=8)
+    Wt = gu.bf16_from_bits(Wb)
+    if group:
+        packed, S, Z = wq.wq_quantize_rtn_g128(Wt, 4, group, True)
+    else:
+        packed, S, Z = wq.wq_quantize_rtn_per_tensor(Wt)
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, group)
+    assert wq.wq_get_status() == 0
+    W64 = wq_inputs.bf16_bits_to_f64(Wb)
+    rows = _sampled_rows(4096, 128, 11 + group)
+    if group:
+        codes, So, Zo = oracle.quantize_rtn_asym(W64[rows], group)
+        np.testing.assert_array_equal(gu.to_np(packed)[rows], oracle.pack_int4(codes))
+        np.testing.assert_array_equal(gu.bits16(S)[rows].ravel(), gu.f16_bits_of(So).ravel())
+        np.testing.assert_array_equal(gu.bits16(Z)[rows].ravel(), gu.f16_bits_of(Zo).ravel())
+    else:
+        codes_all, So, Zo = oracle.quantize_rtn_asym(W64, 0)
+        np.testing.assert_array_equal(gu.to_np(packed), oracle.pack_int4(codes_all))
+        np.testing.assert_array_equal(gu.bits16(S).ravel(), gu.f16_bits_of(So).ravel())
+        np.testing.assert_array_equal(gu.bits16(Z).ravel(), gu.f16_bits_of(Zo).ravel())
+        codes = codes_all[rows]
+    What = oracle.dequant_asym(codes, So, Zo, group)
+    Yref = oracle.matmul_f64(wq_inputs.bf16_bits_to_f64(Xb), What)
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref) <= GATE
+
+
+@pytest.mark.parametrize("N,K,group", [(77, 1120, 32), (80, 1120, 32), (77, 1120, 0)])
+def test_m1_fallback_kernels(N, K, group):
+    """M = 1 shapes that none of the tiled decode kernels take (K not a multiple of 128, N not
+    a multiple of 16): the register-fed kernels, by rows of 8 (N = 80) or not (N = 77)."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + K + group)
+    Xb = wq_inputs.act_bf16(1, K, seed=3)
+    packed, S, Z, codes, So, Zo = _quantize_both(Wb, group)
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, group)
+    assert wq.wq_get_status() == 0
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, group, "exact")
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE

@@ -18,6 +18,7 @@ torch = pytest.importorskip("torch")
 if not torch.cuda.is_available():  # pragma: no cover
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
+import oracle  # noqa: E402
 import w4a16_dequant_matmul_b200 as wq  # noqa: E402
 import wq_inputs  # noqa: E402
 
@@ -27,8 +28,9 @@ def _noalloc_via_c_abi(W):
     packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
     S = torch.empty((1,), dtype=torch.float16, device=W.device)
     Z = torch.empty((1,), dtype=torch.float16, device=W.device)
+    dt = wq.WQ_F32 if W.dtype == torch.float32 else wq.WQ_BF16
     st = wq.lib().wq_quantize_rtn_per_tensor_noalloc(
-        ctypes.c_void_p(W.data_ptr()), wq.WQ_BF16, N, K, W.stride(0),
+        ctypes.c_void_p(W.data_ptr()), dt, N, K, W.stride(0),
         ctypes.c_void_p(packed.data_ptr()), ctypes.c_void_p(S.data_ptr()),
         ctypes.c_void_p(Z.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0, wq.status_name(st)
@@ -46,3 +48,16 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert torch.equal(p0, p1)
         assert torch.equal(s0.view(torch.int16), s1.view(torch.int16))
         assert torch.equal(z0.view(torch.int16), z1.view(torch.int16))
+
+
+def test_noalloc_fp32_weights_match_the_oracle():
+    """fp32 weights through the library's scratch array: codes, S and Z equal the oracle's
+    per-tensor quantization bit for bit, on two calls in a row."""
+    for seed, sigma in ((31, 0.02), (32, 3.0)):
+        W = np.random.default_rng(seed).normal(0, sigma, (200, 1024)).astype(np.float32)
+        W[7, 100] *= 40.0  # one outlier sets the tensor-wide range
+        p, s_, z = _noalloc_via_c_abi(torch.from_numpy(W).cuda())
+        assert wq.wq_get_status() == 0
+        codes, So, Zo = oracle.quantize_rtn_asym(W.astype(np.float64), 0)
+        np.testing.assert_array_equal(p.cpu().numpy(), oracle.pack_int4(codes))
+        assert float(s_.float().item()) == So[0, 0] and float(z.float().item()) == Zo[0, 0]

@@ -17,6 +17,7 @@ S and Z are returned as torch.float16 tensors (binary16 bit patterns in the C AB
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -35,7 +36,7 @@ WQ_F32, WQ_BF16, WQ_F16, WQ_U8, WQ_I8 = 0, 1, 2, 3, 4
 STATUS_NAMES = {
     0: "WQ_OK", 1: "WQ_ERR_NULL", 2: "WQ_ERR_SHAPE", 3: "WQ_ERR_ALIGN", 4: "WQ_ERR_DTYPE",
     5: "WQ_ERR_UNSUPPORTED", 6: "WQ_ERR_CUDA", 7: "WQ_ERR_NONFINITE", 8: "WQ_ERR_TIMEOUT",
-    9: "WQ_ERR_RANGE", 10: "WQ_ERR_NODEVICE",
+    9: "WQ_ERR_RANGE", 10: "WQ_ERR_NODEVICE", 11: "WQ_ERR_DEVICE",
 }
 
 
@@ -134,6 +135,26 @@ def _stream_handle(t, stream=None) -> int:
     return _RAW_STREAM(dev)
 
 
+_GET_DEVICE = None
+
+
+def _on_device(t):
+    """A context that makes the CUDA device holding tensor t current for the call (the C
+    library works on the current device and rejects other devices' memory); a no-op when
+    it already is current, or when t is not a CUDA tensor."""
+    global _GET_DEVICE
+    d = t.get_device()
+    if d < 0:
+        return contextlib.nullcontext()
+    import torch
+
+    if _GET_DEVICE is None:
+        _GET_DEVICE = getattr(torch._C, "_cuda_getDevice", None) or torch.cuda.current_device
+    if _GET_DEVICE() == d:
+        return contextlib.nullcontext()
+    return torch.cuda.device(d)
+
+
 def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
@@ -182,8 +203,9 @@ def wq_quantize_rtn_g128(W, w_bit: int = 4, group: int = 128, zero_point: bool =
         packed = torch.empty((N, K), dtype=torch.int8, device=dev) if packed is None else packed
         S = torch.empty((N,), dtype=torch.float16, device=dev) if S is None else S
     p = _QParams(w_bit, group, 1 if zero_point else 0)
-    st = lib().wq_quantize_rtn_g128(_ptr(W), _w_dtype(W), N, K, ldw, ctypes.byref(p),
-                                    _ptr(packed), _ptr(S), _ptr(Z), _stream(stream))
+    with _on_device(W):
+        st = lib().wq_quantize_rtn_g128(_ptr(W), _w_dtype(W), N, K, ldw, ctypes.byref(p),
+                                        _ptr(packed), _ptr(S), _ptr(Z), _stream(stream))
     _check(st, "wq_quantize_rtn_g128")
     return packed, S, Z
 
@@ -205,10 +227,11 @@ def wq_quantize_rtn_per_tensor(W, workspace=None, stream=None):
     nbytes = wq_quantize_per_tensor_workspace_bytes(N, K)
     if workspace is None:
         workspace = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
-    st = lib().wq_quantize_rtn_per_tensor(_ptr(W), _w_dtype(W), N, K, ldw, _ptr(packed),
-                                          _ptr(S), _ptr(Z), _ptr(workspace),
-                                          workspace.numel() * workspace.element_size(),
-                                          _stream(stream))
+    with _on_device(W):
+        st = lib().wq_quantize_rtn_per_tensor(_ptr(W), _w_dtype(W), N, K, ldw, _ptr(packed),
+                                              _ptr(S), _ptr(Z), _ptr(workspace),
+                                              workspace.numel() * workspace.element_size(),
+                                              _stream(stream))
     _check(st, "wq_quantize_rtn_per_tensor")
     return packed, S, Z
 
@@ -225,8 +248,10 @@ def wq_quantize_rtn_per_tensor_noalloc(W, stream=None):
     packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
     S = torch.empty((1,), dtype=torch.float16, device=W.device)
     Z = torch.empty((1,), dtype=torch.float16, device=W.device)
-    st = lib().wq_quantize_rtn_per_tensor_noalloc(_ptr(W), _w_dtype(W), N, K, ldw, _ptr(packed),
-                                                  _ptr(S), _ptr(Z), _stream(stream))
+    with _on_device(W):
+        st = lib().wq_quantize_rtn_per_tensor_noalloc(_ptr(W), _w_dtype(W), N, K, ldw,
+                                                      _ptr(packed), _ptr(S), _ptr(Z),
+                                                      _stream(stream))
     _check(st, "wq_quantize_rtn_per_tensor_noalloc")
     return packed, S, Z
 
@@ -239,7 +264,9 @@ def wq_pack_int4(codes, packed=None, stream=None):
     if not codes.is_contiguous():
         raise ValueError("codes must be contiguous")
     packed = torch.empty((N, K // 2), dtype=torch.uint8, device=codes.device) if packed is None else packed
-    _check(lib().wq_pack_int4(_ptr(codes), N, K, _ptr(packed), _stream(stream)), "wq_pack_int4")
+    with _on_device(codes):
+        st = lib().wq_pack_int4(_ptr(codes), N, K, _ptr(packed), _stream(stream))
+    _check(st, "wq_pack_int4")
     return packed
 
 
@@ -252,8 +279,10 @@ def wq_dequant(packed, S, Z, group: int = 128, out_dtype=None, out=None, stream=
     K = 2 * K2
     code = WQ_F32 if out_dtype == torch.float32 else WQ_BF16 if out_dtype == torch.bfloat16 else -1
     out = torch.empty((N, K), dtype=out_dtype, device=packed.device) if out is None else out
-    _check(lib().wq_dequant(_ptr(packed), _ptr(S), _ptr(Z), N, K, group, _ptr(out), code,
-                            _stream(stream)), "wq_dequant")
+    with _on_device(packed):
+        st = lib().wq_dequant(_ptr(packed), _ptr(S), _ptr(Z), N, K, group, _ptr(out), code,
+                              _stream(stream))
+    _check(st, "wq_dequant")
     return out
 
 
@@ -274,8 +303,9 @@ def wq_w4a16_gemm(X, packed, S, Z, group: int = 128, Y=None, stream=None):
 
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
     ldy = _rows(Y, "Y")
-    st = _GEMM(X.data_ptr(), M, ldx, packed.data_ptr(), S.data_ptr(), Z.data_ptr(), N, K, group,
-               Y.data_ptr(), ldy, _stream_handle(X, stream))
+    with _on_device(X):
+        st = _GEMM(X.data_ptr(), M, ldx, packed.data_ptr(), S.data_ptr(), Z.data_ptr(), N, K,
+                   group, Y.data_ptr(), ldy, _stream_handle(X, stream))
     if st != 0:
         raise WQError(st, "wq_w4a16_gemm")
     return Y
@@ -290,8 +320,10 @@ def wq_w8a16_gemm(X, codes, S, Y=None, stream=None):
     ldx = _rows(X, "X")
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device) if Y is None else Y
     ldy = _rows(Y, "Y")
-    _check(lib().wq_w8a16_gemm(_ptr(X), M, ldx, _ptr(codes), _ptr(S), N, K, _ptr(Y), ldy,
-                               _stream(stream)), "wq_w8a16_gemm")
+    with _on_device(X):
+        st = lib().wq_w8a16_gemm(_ptr(X), M, ldx, _ptr(codes), _ptr(S), N, K, _ptr(Y), ldy,
+                                 _stream(stream))
+    _check(st, "wq_w8a16_gemm")
     return Y
 
 

@@ -1,5 +1,6 @@
 // C ABI of libwq (declared in include/wq.h): argument validation, kernel choice by shape,
 // the device status word. No device memory is allocated here.
+#include <initializer_list>
 #include <mutex>
 
 #include "../../include/wq.h"
@@ -13,36 +14,62 @@ __device__ unsigned g_wq_status;  // per-device status word (bits wq::kSt*)
 
 constexpr int kMaxDevices = 64;
 struct DeviceInfo {
-  bool ready = false;
-  bool ok = false;
+  bool ok = false;             // set once the queries below have succeeded
   int sms = 0;
   unsigned* status = nullptr;  // device address of g_wq_status on that device
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
-// Current device's cached info (SM count, status-word address); nullptr if unusable.
+// Current device's cached info (SM count, status-word address); nullptr if unusable. Only
+// a successful set of queries is kept: a failure (no device, not sm_100, a lookup refused
+// during a stream capture) is returned as is and retried by the next call.
 const DeviceInfo* device_info() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
   std::lock_guard<std::mutex> lock(g_dev_mu);
   DeviceInfo& d = g_dev[dev];
-  if (!d.ready) {
-    d.ready = true;
-    int major = 0, minor = 0;
+  if (!d.ok) {
+    int major = 0, minor = 0, sms = 0;
     void* addr = nullptr;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
         major == 10 && minor == 0 && cudaGetSymbolAddress(&addr, g_wq_status) == cudaSuccess) {
+      d.sms = sms;
       d.status = static_cast<unsigned*>(addr);
       d.ok = true;
+    } else {
+      cudaGetLastError();
     }
   }
   return d.ok ? &d : nullptr;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Every non-null pointer is device memory of the current device, or managed memory.
+bool on_current_device(std::initializer_list<const void*> ptrs) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  for (const void* p : ptrs) {
+    if (!p) continue;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    if (at.type == cudaMemoryTypeManaged) continue;
+    if (at.type != cudaMemoryTypeDevice || at.device != dev) return false;
+  }
+  return true;
+}
 
 wq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
 
@@ -51,6 +78,10 @@ bool fits_int(int64_t v) { return v >= 0 && v <= 0x7fffffffLL; }
 }  // namespace
 
 namespace wq {
+bool pointers_on_current_device(std::initializer_list<const void*> ptrs) {
+  return on_current_device(ptrs);
+}
+
 bool current_device(int* sms, unsigned** status) {
   const DeviceInfo* d = device_info();
   if (!d) return false;
@@ -77,6 +108,7 @@ const char* wq_status_string(wq_status s) {
     case WQ_ERR_TIMEOUT: return "device wait timed out";
     case WQ_ERR_RANGE: return "code out of range [0, 15]";
     case WQ_ERR_NODEVICE: return "no usable sm_100 CUDA device";
+    case WQ_ERR_DEVICE: return "a pointer is not memory of the current device";
   }
   return "unknown status";
 }
@@ -102,6 +134,7 @@ wq_status wq_quantize_rtn_g128(const void* W, wq_dtype w_dtype, int64_t N, int64
     return WQ_ERR_ALIGN;
   const DeviceInfo* d = device_info();
   if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({W, packed, S, Z})) return WQ_ERR_DEVICE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf16 = w_dtype == WQ_BF16;
   if (int4)
@@ -134,6 +167,7 @@ wq_status wq_quantize_rtn_per_tensor(const void* W, wq_dtype w_dtype, int64_t N,
     return WQ_ERR_ALIGN;
   const DeviceInfo* d = device_info();
   if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({W, packed, S, Z, workspace})) return WQ_ERR_DEVICE;
   const int nparts = wq::per_tensor_parts(d->sms);
   if (workspace_bytes < static_cast<size_t>(nparts) * sizeof(float2)) return WQ_ERR_SHAPE;
   return from_cuda(wq::launch_quant_per_tensor(
@@ -150,6 +184,7 @@ wq_status wq_pack_int4(const uint8_t* codes, int64_t N, int64_t K, uint8_t* pack
   if (!aligned(codes, 16) || !aligned(packed, 16)) return WQ_ERR_ALIGN;
   const DeviceInfo* d = device_info();
   if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({codes, packed})) return WQ_ERR_DEVICE;
   return from_cuda(wq::launch_pack_int4(codes, N, K, packed, d->status, d->sms,
                                         static_cast<cudaStream_t>(stream)));
 }
@@ -166,6 +201,7 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
     return WQ_ERR_ALIGN;
   const DeviceInfo* d = device_info();
   if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({packed, S, Z, out})) return WQ_ERR_DEVICE;
   const int g = group ? group : (int)K;
   const int sz_row = group ? (int)(K / group) : 0;
   return from_cuda(wq::launch_dequant(packed, S, Z, N, (int)K, g, sz_row, out,
@@ -192,6 +228,7 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
     return WQ_ERR_ALIGN;
   const DeviceInfo* d = device_info();
   if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({X, packed, S, Z, Y})) return WQ_ERR_DEVICE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int g = group ? group : (int)K;
   const int sz_row = group ? (int)(K / group) : 0;
@@ -199,7 +236,7 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
                  ldy, d->status};
   // M = 1 beyond the register-loaded kernels' K only where the streaming kernel takes it
   if (M <= kSkinnyMaxM &&
-      (M > 1 || K <= wq::gemv_max_k() || wq::gemv_tma_ok(a) ||
+      (M > 1 || K <= wq::gemv_max_k() || wq::gemv_imma_bulk_ok(a) || wq::gemv_tma_ok(a) ||
        (wq::gemv_stream_ok(a) && wq::gemv_stream_fits(a)))) {
     // Small M: the decode kernels, in passes over blocks of tokens when the whole of M has
     // no fast kernel (the weights come from HBM once; later passes find them in L2).
@@ -237,6 +274,7 @@ wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t*
     return WQ_ERR_ALIGN;
   const DeviceInfo* d = device_info();
   if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({X, codes, S, Y})) return WQ_ERR_DEVICE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (M <= 8) {
     wq::Gemv8Args a{X, ldx, codes, S, (int)M, (int)N, (int)K, Y, ldy};

@@ -15,6 +15,18 @@
 
 namespace wq {
 
+// Let kernel `kern` use `bytes` of dynamic shared memory, with all of the SM's unified L1 /
+// shared memory configured as shared memory. Every large-shared-memory kernel of the library
+// asks for the same split, so consecutive launches of different kernels on a stream do not
+// make an SM change its split between them (which needs the SM to drain first).
+template <typename F>
+inline cudaError_t set_smem_attrs(F* kern, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  return e;
+}
+
 // Bits of the device status word (see wq_get_status).
 enum : unsigned { kStNonFinite = 1u, kStRange = 2u, kStTimeout = 4u };
 

@@ -4,9 +4,9 @@
 // at decode the matmul is bound by the bytes of weights read from memory.)
 //
 // Work: tiles of 16 weight rows; a CTA owns a contiguous range of tiles, the same number
-// for every CTA (the grid is sized so). Each tile's rows are streamed in K-chunks of at
-// least 2 KB per row (whole rows up to 3 KB): on B200 the bulk-copy engine keeps about 32
-// copies in flight per SM, so copies this large are what fills HBM.
+// for every CTA (the grid is sized so). Each tile's rows are streamed whole (up to 3 KB per
+// row, K <= 6144; longer rows go to the K-chunked TMA kernel): on B200 the bulk-copy engine
+// keeps about 32 copies in flight per SM, so copies this large are what fills HBM.
 //
 // Warp roles (one CTA per SM):
 //   producer  one lane. X (one bulk copy per token), then per chunk: 16 row copies into a
@@ -36,6 +36,8 @@
 // Every wait is bounded (2 s): on a timeout the kernel records kStTimeout, the producer
 // waits (bounded) for the copies it issued to land, and all warps return.
 #include <type_traits>
+
+#include <atomic>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -410,6 +412,8 @@ cudaError_t launch_decode_m(const GemvArgs& a, int sms, cudaStream_t st) {
   if (ntiles == 0) return cudaSuccess;
   const int row_bytes = a.K / 2;
   const int NCH = (row_bytes + kChunkMax - 1) / kChunkMax;
+  // whole rows only: rows split into several K-chunks are left to the other kernels
+  if (NCH != 1) return cudaErrorInvalidValue;
   const int CK = static_cast<int>(align_up((row_bytes + NCH - 1) / NCH, 64));
   if ((NCH - 1) * CK >= row_bytes) return cudaErrorInvalidValue;  // no empty last chunk
   const int pitch = CK + ((64 - CK % 128) + 128) % 128;  // = 64 (mod 128)
@@ -427,14 +431,13 @@ cudaError_t launch_decode_m(const GemvArgs& a, int sms, cudaStream_t st) {
   const size_t smem = L.total + slack;
 
   auto kern = gemv_decode<M>;
-  static bool attr[64] = {false};
+  static std::atomic<bool> attr[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!attr[dev & 63]) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(kSmemBudget));
+  if (!attr[dev & 63].load(std::memory_order_acquire)) {
+    const cudaError_t e = set_smem_attrs(kern, static_cast<int>(kSmemBudget));
     if (e != cudaSuccess) return e;
-    attr[dev & 63] = true;
+    attr[dev & 63].store(true, std::memory_order_release);
   }
   const int tpc = (ntiles + sms - 1) / sms;
   const int grid = (ntiles + tpc - 1) / tpc;
@@ -458,6 +461,7 @@ bool gemv_stream_fits(const GemvArgs& a) {
   if (a.M < 1 || a.M > 4 || a.K % 128 != 0) return false;
   const int row_bytes = a.K / 2;
   const int NCH = (row_bytes + kChunkMax - 1) / kChunkMax;
+  if (NCH != 1) return false;  // whole rows only (K <= 6144)
   const int CK = static_cast<int>(align_up((row_bytes + NCH - 1) / NCH, 64));
   if ((NCH - 1) * CK >= row_bytes) return false;
   const int pitch = CK + ((64 - CK % 128) + 128) % 128;

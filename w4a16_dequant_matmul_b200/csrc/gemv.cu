@@ -19,6 +19,8 @@
 //
 // gemv_rows<M> (2 <= M <= 8): one warp per output row, X re-read through L1; a simple
 //   path for small batches.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -844,7 +846,7 @@ cudaError_t launch_m1_bulk(const GemvArgs& a, int sms, cudaStream_t st) {
   Cfg& c = cache[dev & 63][(a.K / 32 + G) & 7];
   const int key = a.K * 4096 + G;
   if (c.key != key) {
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    set_smem_attrs(kern, 200 * 1024);
     int stages = static_cast<int>((100 * 1024 - fixed) / stage);
     if (stages > 8) stages = 8;
     int occ = 0;
@@ -882,7 +884,7 @@ cudaError_t launch_mma(const GemvArgs& a, int sms, cudaStream_t st) {
   cudaGetDevice(&dev);
   int& occ = occ_cache[dev & 63];
   if (occ == 0) {
-    cudaFuncSetAttribute(gemv_mma<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    set_smem_attrs(gemv_mma<M>, 96 * 1024);
     occ = -1;
   }
   int o = 0;
@@ -907,13 +909,12 @@ cudaError_t launch_mma_bulk(const GemvArgs& a, int sms, cudaStream_t st) {
   if (stages < 2) return cudaErrorInvalidValue;
   const size_t smem = MmaBulkLayout(M, a.K, wstride, stages, NW, RT).total;
   auto kern = gemv_mma_bulk<M, NW, RT>;
-  static bool attr[64] = {false};
+  static std::atomic<bool> attr[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!attr[dev & 63]) {
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(kBudget));
-    attr[dev & 63] = true;
+  if (!attr[dev & 63].load(std::memory_order_acquire)) {
+    set_smem_attrs(kern, static_cast<int>(kBudget));
+    attr[dev & 63].store(true, std::memory_order_release);
   }
   const int ntiles = a.N / (16 * RT);
   const int grid = ntiles < sms ? ntiles : sms;
@@ -996,7 +997,7 @@ int gemv_fast_block(const GemvArgs& a) {
     if (b > a.M || b > 8) continue;
     GemvArgs t = a;
     t.M = b;
-    if (bulk_fits(b) || gemv_stream_fits(t) || gemv_tma_ok(t)) return b;
+    if (bulk_fits(b) || gemv_stream_fits(t) || gemv_tma_ok(t) || gemv_imma_bulk_ok(t)) return b;
   }
   return 0;
 }
@@ -1009,6 +1010,12 @@ static bool mma_bulk_rt2_fits(const GemvArgs& a) {
 }
 
 cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st) {
+  // M <= 2, g = 128, short rows: the integer-MMA kernel on whole-row tiles (gemv_imma.cu)
+  // where two stages of them fit in shared memory.
+  if (a.M <= 2 && gemv_imma_bulk_ok(a)) {
+    const cudaError_t e = launch_gemv_imma_bulk(a, sms, st);
+    if (e != cudaErrorInvalidValue) return e;
+  }
   // M <= 4 with long rows (two whole 32-row tiles do not fit the bulk-copy kernel's shared
   // memory): the TMA-fed kernel that streams 32-row tiles in K chunks (N % 32 == 0).
   // Otherwise M = 1: the bulk-copy kernel (whole rows; measured fastest for short rows);

@@ -6,28 +6,32 @@
 // at decode the matmul is bound by the bytes of weights read from memory.)
 //
 // Work: tiles of 32 weight rows; a CTA (one per SM) owns a contiguous, balanced range of them.
-// A tile streams in chunks of CG = 32, 16 or 8 groups (the largest whose ring has two stages):
-// one TMA box of 64 bytes x 32 rows x CG groups that lands as [group][row][64 B], so the two
-// rows a quarter-warp reads sit 64 bytes apart and its 16-byte loads cover all 32 banks. The
-// tile's S' and Z (32 x G each, contiguous in HBM) arrive by two bulk copies into a slot of
-// their own. Before it waits for the previous kernel (programmatic dependent launch), each CTA
-// warms L2 with its codes past the first ring's worth (hints only, so safe before the wait).
+// A tile streams in chunks of CG = 32, 16 or 8 groups (the largest whose ring fits): one TMA
+// box of 64 bytes x 32 rows x CG groups that lands as [group][row][64 B], so the two rows a
+// quarter-warp reads sit 64 bytes apart and its 16-byte loads cover all 32 banks. The tile's
+// S' and Z (32 x G each, contiguous in HBM) arrive by two bulk copies into a slot of their own.
+// X is copied into shared memory first, when that leaves at least 64 KB of ring; otherwise it
+// is read from global memory once, up front. Before it waits for the previous kernel
+// (programmatic dependent launch), each CTA warms L2 with its codes past the first ring's
+// worth (hints only, so safe before the wait).
 //
 // Warp roles:
-//   producer  one lane: X (one bulk copy per token), then per tile the S'/Z copies and the
-//             chunk boxes into the stage ring.
+//   producer  one lane: X, then per tile the S'/Z copies and the chunk boxes into the ring.
 //   consumers 16 warps. Every warp takes every chunk and its share of the chunk's groups, so
 //             each warp waits for every fill of every stage in order (the parity waits
-//             cannot alias). Per group a warp reads the X fragments once and multiplies both
-//             16-row halves of the tile: codes decoded to bf16 (1 + q/16), eight m16n8k16
-//             MMAs per half in four accumulator chains, and with D = sum x (1 + q/16),
-//               acc += S' (16 D - (16 + Z) sum x).
+//             cannot alias). The arithmetic is the integer warp-level MMA of imma_digits.cuh:
+//             per group a warp prepares the digit fragments of X once (only that warp reads
+//             them), then multiplies both 16-row halves of the tile against one load of
+//             them, exactly in integers, and applies S' and the group's scale in fp32.
 //   epilogue  sums the 16 warps' partials of a tile in warp order (deterministic) and writes
 //             Y in bf16.
 // Every wait is bounded (2 s): on a timeout the kernel records kStTimeout, the producer waits
 // (bounded) for the copies it issued, and all warps return.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "imma_digits.cuh"
 #include "mma_frag.cuh"
 #include "ptx.cuh"
 #include "tma_host.h"
@@ -39,7 +43,6 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kNW = 16;                          // consumer warps
 constexpr int kTR = 32;                          // weight rows per tile
 constexpr int kMaxCG = 32;                       // groups per chunk, at most (64 KB)
-constexpr int kSzSlots = 2;                      // tiles of S'/Z in flight
 constexpr int kPartSlots = 2;                    // tiles between consumers and epilogue
 constexpr int kMaxStages = 8;
 constexpr int kThreads = 32 * (kNW + 2);
@@ -51,27 +54,41 @@ __host__ __device__ constexpr uint32_t align_up(uint32_t v, uint32_t a) { return
 
 // Shared-memory layout (byte offsets from a 128-aligned base; host and device agree).
 struct TmaLayout {
-  uint32_t xf, xsp, sx, sz, sz_slot, part, part_slot, ring, bar, total;
-  __host__ __device__ TmaLayout(int M, int G, int NS, int CG) {
+  uint32_t xraw, frag, xs, xp, xf, xsp, sx, sz, sz_slot, part, part_slot, ring, bar, total;
+  __host__ __device__ TmaLayout(int M, int G, int NS, int CG, bool kInt, bool x_staged,
+                                int sz_slots) {
     const uint32_t MR = M < 2 ? 2 : M;
-    xf = 0;                                  // [M][G][4][16] u32 X fragments
-    xsp = xf + G * 4u * M * 64;              // [M][G][4] f32 partial sums of x
-    sx = xsp + G * 4u * M * 4;               // [G][8] f32 sums of x per token
-    sz = align_up(sx + G * 32u, 128);
+    const uint32_t NB = (4 * M + 7) / 8, FC = M == 1 ? 3 : 8;
+    uint32_t end;
+    xraw = xf = xsp = sx = frag = xs = xp = 0;
+    if (kInt) {
+      xraw = 0;                                      // [M][K] bf16: X as copied (if staged)
+      frag = xraw + (x_staged ? M * G * 256u : 0u);  // [G][NB * FC * 128] digit fragments
+      xs = align_up(frag + G * NB * FC * 128, 16);   // [G][NB * 8] f32 column sums
+      xp = xs + G * NB * 32u;                        // [G][M] f32 scales 2^-s
+      end = xp + G * M * 4u;
+    } else {
+      xf = 0;                                  // [M][G][4][16] u32 X fragments (bf16 MMA)
+      xsp = xf + G * 4u * M * 64;              // [M][G][4] f32 partial sums of x
+      sx = xsp + G * 4u * M * 4;               // [G][8] f32 sums of x per token
+      end = sx + G * 32u;
+    }
+    sz = align_up(end, 128);
     sz_slot = align_up(128u * G, 128);       // S' [32][G] u16, then Z [32][G] u16
-    part = sz + kSzSlots * sz_slot;
+    part = sz + sz_slots * sz_slot;
     part_slot = kNW * kTR * MR * 4;          // [16 warps][32 rows][MR] f32
     ring = align_up(part + kPartSlots * part_slot, 128);
     bar = ring + NS * (kTR * 64u * CG);
-    total = bar + (2u * NS + 2u * kSzSlots + 2u * kPartSlots + 1u) * 8;
+    total = bar + (2u * NS + 2u * sz_slots + 2u * kPartSlots + 1u) * 8;
   }
 };
 
-template <int M>
+template <int M, bool kInt>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X, int64_t ldx,
          const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int N, int K, int NS,
-         int CG, int prefetch_tiles, uint16_t* __restrict__ Y, int64_t ldy, unsigned* status) {
+         int CG, int x_staged, int sz_slots, int prefetch_tiles, uint16_t* __restrict__ Y,
+         int64_t ldy, unsigned* status) {
   constexpr int MR = M < 2 ? 2 : M;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
@@ -79,12 +96,12 @@ gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X
   const int G = K / 128;
   const int NCH = (G + CG - 1) / CG;
   const uint32_t stage = kTR * 64u * CG;  // bytes of one chunk
-  const TmaLayout L(M, G, NS, CG);
+  const TmaLayout L(M, G, NS, CG, kInt, x_staged != 0, sz_slots);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint64_t* empty = full + NS;
   uint64_t* szfull = empty + NS;
-  uint64_t* szempty = szfull + kSzSlots;
-  uint64_t* tdone = szempty + kSzSlots;
+  uint64_t* szempty = szfull + sz_slots;
+  uint64_t* tdone = szempty + sz_slots;
   uint64_t* pempty = tdone + kPartSlots;
   uint64_t* xfull = pempty + kPartSlots;
   const int warp = threadIdx.x >> 5;
@@ -100,7 +117,7 @@ gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kNW);
     }
-    for (int i = 0; i < kSzSlots; ++i) {
+    for (int i = 0; i < sz_slots; ++i) {
       mbar_init(&szfull[i], 1);
       mbar_init(&szempty[i], kNW);
     }
@@ -126,15 +143,17 @@ gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X
 
   if (warp == kNW) {  // ---------------------------------------------------------- producer
     if (lane != 0) return;
-    mbar_arrive_expect_tx(xfull, static_cast<uint32_t>(M) * K * 2);
-    for (int n = 0; n < M; ++n)
-      bulk_g2s(smem + L.xf + static_cast<uint32_t>(n) * K * 2, X + n * ldx, K * 2u, xfull);
+    if (!kInt || x_staged) {  // X first, so that it lands ahead of the weights
+      mbar_arrive_expect_tx(xfull, static_cast<uint32_t>(M) * K * 2);
+      for (int n = 0; n < M; ++n)
+        bulk_g2s(smem + L.xraw + static_cast<uint32_t>(n) * K * 2, X + n * ldx, K * 2u, xfull);
+    }
     int i = 0, tl = 0;
     bool ok = true;
     for (; tl < my_tiles && ok; ++tl) {
-      const int tile = t_begin + tl, ss = tl % kSzSlots;
-      if (tl >= kSzSlots &&
-          !mbar_wait_spin_bounded(&szempty[ss], ((tl / kSzSlots) - 1) & 1u, kWaitNs)) {
+      const int tile = t_begin + tl, ss = tl % sz_slots;
+      if (tl >= sz_slots &&
+          !mbar_wait_spin_bounded(&szempty[ss], ((tl / sz_slots) - 1) & 1u, kWaitNs)) {
         set_status(status, kStTimeout);
         break;
       }
@@ -158,10 +177,11 @@ gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X
     for (int st = 0; st < NS && st < i; ++st)
       if (!mbar_wait_spin_bounded(&full[st], ((i - 1 - st) / NS) & 1u, kWaitNs))
         set_status(status, kStTimeout);
-    for (int ss = 0; ss < kSzSlots && ss < tl; ++ss)
-      if (!mbar_wait_spin_bounded(&szfull[ss], ((tl - 1 - ss) / kSzSlots) & 1u, kWaitNs))
+    for (int ss = 0; ss < sz_slots && ss < tl; ++ss)
+      if (!mbar_wait_spin_bounded(&szfull[ss], ((tl - 1 - ss) / sz_slots) & 1u, kWaitNs))
         set_status(status, kStTimeout);
-    if (!mbar_wait_spin_bounded(xfull, 0, kWaitNs)) set_status(status, kStTimeout);
+    if ((!kInt || x_staged) && !mbar_wait_spin_bounded(xfull, 0, kWaitNs))
+      set_status(status, kStTimeout);
     return;
   }
 
@@ -188,6 +208,181 @@ gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X
     return;
   }
 
+  if constexpr (kInt) {
+  // ---------------------------------------------------------------------- consumer warps
+  // Warp w takes, of every chunk, the groups [qa, qb) of its even share. Before the first
+  // tile's chunk ch is consumed it turns the X of its groups of chunk ch + 1 into digit
+  // fragments (imma_digits.cuh; only this warp reads them), so that work overlaps the wait.
+  using C = Cols<M>;
+  constexpr int NB = C::NB, FC = C::FC;
+  auto share = [&](int ch, int& ga, int& gb) {  // this warp's groups of chunk ch
+    const int g0 = ch * CG, gn = min(CG, G - g0);
+    ga = g0 + (warp * gn) / kNW;
+    gb = g0 + ((warp + 1) * gn) / kNW;
+  };
+  auto prep_one = [&](int gi, const uint2 (&xv)[M]) {
+    prep_group<M>(smem + L.frag + gi * C::kFragBytes,
+                  reinterpret_cast<float*>(smem + L.xs) + gi * NB * 8,
+                  reinterpret_cast<float*>(smem + L.xp) + gi * M, xv, lane);
+  };
+  auto prep_chunk = [&](int ch) {  // from the staged copy of X
+    int ga, gb;
+    share(ch, ga, gb);
+    for (int gi = ga; gi < gb; ++gi) {
+      uint2 xv[M];
+#pragma unroll
+      for (int m = 0; m < M; ++m)
+        xv[m] = *reinterpret_cast<const uint2*>(smem + L.xraw + (m * G + gi) * 256 + 8 * lane);
+      prep_one(gi, xv);
+    }
+    __syncwarp();
+  };
+  if (x_staged) {
+    if (!mbar_wait_spin_bounded(xfull, 0, kWaitNs)) {
+      set_status(status, kStTimeout);
+      return;
+    }
+    prep_chunk(0);
+  } else {
+    // X from global memory, all of this warp's groups at once: the loads of a batch are all
+    // issued before any is used, so their latency is paid once per batch
+    constexpr int BG = 16 / M;
+    int gl[BG];
+    int n = 0;
+    auto flush = [&]() {
+      uint2 xv[BG][M];
+#pragma unroll
+      for (int u = 0; u < BG; ++u)
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+          xv[u][m] = u < n ? *reinterpret_cast<const uint2*>(X + m * ldx + gl[u] * 128 + 4 * lane)
+                           : make_uint2(0u, 0u);
+#pragma unroll
+      for (int u = 0; u < BG; ++u)
+        if (u < n) prep_one(gl[u], xv[u]);
+      n = 0;
+    };
+    for (int ch = 0; ch < NCH; ++ch) {
+      int ga, gb;
+      share(ch, ga, gb);
+      for (int gi = ga; gi < gb; ++gi) {
+        gl[n++] = gi;
+        if (n == BG) flush();
+      }
+    }
+    if (n > 0) flush();
+    __syncwarp();
+  }
+  const float* xs_all = reinterpret_cast<const float*>(smem + L.xs);
+  const float* xp_all = reinterpret_cast<const float*>(smem + L.xp);
+  const int r = lane >> 2, c = lane & 3;
+  const float w0 = (c & 1) ? 65536.0f : 1.0f, w1 = (c & 1) ? 16777216.0f : 256.0f;
+  const bool bcol = r < FC;  // this lane's B column is stored (else its digits are zero)
+  const uint32_t ring_lane = base_s + L.ring + r * 64 + 16 * c;
+  uint32_t mask4 = 0x0F0F0F0Fu;
+  asm volatile("" : "+r"(mask4));
+  int i = 0;
+  for (int tl = 0; tl < my_tiles; ++tl) {
+    const int ss = tl % sz_slots, ps = tl % kPartSlots;
+    const uint32_t sb = base_s + L.sz + ss * L.sz_slot, zb = sb + szbytes;
+    float acc[2][NB][2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) acc[t][nb][0] = acc[t][nb][1] = 0.0f;
+    for (int ch = 0; ch < NCH; ++ch, ++i) {
+      const int st = i % NS;
+      if (x_staged && tl == 0 && ch + 1 < NCH) prep_chunk(ch + 1);
+      bool ok = mbar_wait_spin_bounded(&full[st], (i / NS) & 1u, kWaitNs);
+      if (ok && ch == 0) ok = mbar_wait_spin_bounded(&szfull[ss], (tl / sz_slots) & 1u, kWaitNs);
+      if (!ok) {
+        set_status(status, kStTimeout);
+        return;
+      }
+      const uint32_t wst = ring_lane + st * stage;
+      int ga, gb;
+      share(ch, ga, gb);
+      for (int g = ga; g < gb; ++g) {
+        const int q = g - ch * CG;
+        const uint32_t frag_s = base_s + L.frag + g * C::kFragBytes;
+        uint32_t bw[NB][8];
+        float2 xsum[NB];
+        float p[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          const uint32_t blk = frag_s + nb * FC * 128 + (r * 4 + c) * 16;
+          uint4 b01 = make_uint4(0u, 0u, 0u, 0u), b23 = b01;
+          if (bcol) {
+            b01 = lds128(blk);
+            b23 = lds128(blk + FC * 64);
+          }
+          bw[nb][0] = b01.x; bw[nb][1] = b01.y; bw[nb][2] = b01.z; bw[nb][3] = b01.w;
+          bw[nb][4] = b23.x; bw[nb][5] = b23.y; bw[nb][6] = b23.z; bw[nb][7] = b23.w;
+          xsum[nb] = *reinterpret_cast<const float2*>(xs_all + g * NB * 8 + nb * 8 + 2 * c);
+          const int m = 2 * nb + (c >> 1);
+          p[nb] = m < M ? xp_all[g * M + (m < M ? m : 0)] : 0.0f;
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t wa = wst + q * (kTR * 64) + t * (16 * 64);
+          const uint4 ca = lds128(wa);
+          const uint4 cb = lds128(wa + 8 * 64);
+          const int ra = 16 * t + r, rb = ra + 8;
+          const float sa = f16_bits_to_f32(lds16(sb + (ra * G + g) * 2));
+          const float za = f16_bits_to_f32(lds16(zb + (ra * G + g) * 2));
+          const float sbv = f16_bits_to_f32(lds16(sb + (rb * G + g) * 2));
+          const float zbv = f16_bits_to_f32(lds16(zb + (rb * G + g) * 2));
+          const uint32_t wr0[4] = {ca.x, ca.y, ca.z, ca.w};
+          const uint32_t wr1[4] = {cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            // accumulators start at the magic so that each reads back as 1.5 * 2^23 + D
+            int d[4] = {kImmaMagicBits, kImmaMagicBits, kImmaMagicBits, kImmaMagicBits};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint32_t a[4] = {wr0[w] & mask4, wr1[w] & mask4, (wr0[w] >> 4) & mask4,
+                                     (wr1[w] >> 4) & mask4};
+              imma_16832(d, a, bw[nb][2 * w], bw[nb][2 * w + 1]);
+            }
+            // D_i - Z X_i, exactly (both sides carry the same magic offset)
+            const float e0 = __int_as_float(d[0]) - fmaf(za, xsum[nb].x, kImmaMagic);
+            const float e1 = __int_as_float(d[1]) - fmaf(za, xsum[nb].y, kImmaMagic);
+            const float e2 = __int_as_float(d[2]) - fmaf(zbv, xsum[nb].x, kImmaMagic);
+            const float e3 = __int_as_float(d[3]) - fmaf(zbv, xsum[nb].y, kImmaMagic);
+            float va = fmaf(e1, w1, e0 * w0), vb = fmaf(e3, w1, e2 * w0);
+            va += __shfl_xor_sync(0xffffffffu, va, 1);
+            vb += __shfl_xor_sync(0xffffffffu, vb, 1);
+            acc[t][nb][0] = fmaf(sa * p[nb], va, acc[t][nb][0]);
+            acc[t][nb][1] = fmaf(sbv * p[nb], vb, acc[t][nb][1]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    if (lane == 0) mbar_arrive(&szempty[ss]);
+    if (tl >= kPartSlots &&
+        !mbar_wait_spin_bounded(&pempty[ps], ((tl / kPartSlots) - 1) & 1u, kWaitNs)) {
+      set_status(status, kStTimeout);
+      return;
+    }
+    float* part = reinterpret_cast<float*>(smem + L.part + ps * L.part_slot) + warp * kTR * MR;
+    if ((c & 1) == 0) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          const int m = 2 * nb + (c >> 1);
+          if (m < M) {
+            part[(16 * t + r) * MR + m] = acc[t][nb][0];
+            part[(16 * t + r + 8) * MR + m] = acc[t][nb][1];
+          }
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tdone[ps]);
+  }
+  } else {
   // ---------------------------------------------------------------------- consumer warps
   // X (landed in natural order) -> fragment order in place, 64 bytes (32 values of one
   // token, one quarter c of a group) per thread, and per-group token sums, each formed from
@@ -245,13 +440,13 @@ gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X
   asm volatile("" : "+r"(kMask), "+r"(kMagic));
   int i = 0;
   for (int tl = 0; tl < my_tiles; ++tl) {
-    const int ss = tl % kSzSlots, ps = tl % kPartSlots;
+    const int ss = tl % sz_slots, ps = tl % kPartSlots;
     const uint32_t sb = base_s + L.sz + ss * L.sz_slot, zb = sb + szbytes;
     float acc[2][4] = {};
     for (int ch = 0; ch < NCH; ++ch, ++i) {
       const int st = i % NS;
       bool ok = mbar_wait_spin_bounded(&full[st], (i / NS) & 1u, kWaitNs);
-      if (ok && ch == 0) ok = mbar_wait_spin_bounded(&szfull[ss], (tl / kSzSlots) & 1u, kWaitNs);
+      if (ok && ch == 0) ok = mbar_wait_spin_bounded(&szfull[ss], (tl / sz_slots) & 1u, kWaitNs);
       if (!ok) {
         set_status(status, kStTimeout);
         return;
@@ -331,30 +526,49 @@ gemv_tma(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ X
     __syncwarp();
     if (lane == 0) mbar_arrive(&tdone[ps]);
   }
+  }
 }
 
 // Chunk size (groups) and ring depth for this shape: the largest chunk of 32, 16 or 8 groups
 // whose ring has at least two stages in shared memory; NS = 0 if none fits.
 struct TmaCfg {
   int CG, NS;
+  bool x_staged;
+  int sz_slots;
 };
-TmaCfg tma_config(int M, int G) {
-  const uint32_t fixed = TmaLayout(M, G, 0, 8).total + kSlack;
-  for (int cg : {kMaxCG, 16, 8}) {
-    if (fixed > kSmemBudget) break;
-    int ns = static_cast<int>((kSmemBudget - fixed) / (kTR * 64u * cg + 16));
-    if (ns > kMaxStages) ns = kMaxStages;
-    if (ns >= 2) return {cg, ns};
+// Chunk size, ring depth, X staging and S'/Z slots for this shape. The bf16 path takes the
+// largest chunk whose ring has two stages. The integer path also stages X in shared memory
+// (when that leaves at least 64 KB of ring; otherwise X is read once from global memory) and
+// falls back to one S'/Z slot when two leave no ring.
+TmaCfg tma_config(int M, int G, bool kInt) {
+  for (int slots : {2, 1}) {
+    for (bool xs : {true, false}) {
+      if (!kInt && !xs) continue;
+      const uint32_t fixed = TmaLayout(M, G, 0, 8, kInt, xs, slots).total + kSlack;
+      for (int cg : {kMaxCG, 16, 8}) {
+        if (fixed > kSmemBudget) break;
+        int ns = static_cast<int>((kSmemBudget - fixed) / (kTR * 64u * cg + 16));
+        if (ns > kMaxStages) ns = kMaxStages;
+        if (ns >= 2 && (!kInt || !xs || ns * kTR * 64u * cg >= 64u * 1024))
+          return {cg, ns, xs, slots};
+      }
+    }
+    if (!kInt) break;
   }
-  return {8, 0};
+  return {8, 0, false, 2};
 }
 
-template <int M>
-cudaError_t launch_tma_m(const GemvArgs& a, int sms, cudaStream_t st) {
+// The integer MMA for one token while K <= 16384 (G <= 128 groups); beyond that, and for
+// two to four tokens, the digit fragments (3 bytes per k and token, besides the staged X)
+// leave too small a ring and the bf16 MMA, whose X fragments take 2 bytes per k, is faster.
+constexpr int kIntMaxG = 128;
+
+template <int M, bool kInt>
+cudaError_t launch_tma_k(const GemvArgs& a, int sms, cudaStream_t st) {
   const int G = a.K / 128;
   const int ntiles = a.N / kTR;
   if (ntiles == 0) return cudaSuccess;
-  const TmaCfg c = tma_config(M, G);
+  const TmaCfg c = tma_config(M, G, kInt);
   if (c.NS == 0) return cudaErrorInvalidValue;
   // codes as [G groups][N rows][64 bytes]: boxes of CG groups x 32 rows x 64 bytes. The
   // encoded map is kept per thread for the last few weight matrices (decode calls repeat).
@@ -384,16 +598,16 @@ cudaError_t launch_tma_m(const GemvArgs& a, int sms, cudaStream_t st) {
     next_slot = (next_slot + 1) % kMapCache;
     map = &e.map;
   }
-  const size_t smem = TmaLayout(M, G, c.NS, c.CG).total + kSlack;
-  auto kern = gemv_tma<M>;
-  static bool attr[64] = {false};
+  const size_t smem =
+      TmaLayout(M, G, c.NS, c.CG, kInt, c.x_staged, c.sz_slots).total + kSlack;
+  auto kern = gemv_tma<M, kInt>;
+  static std::atomic<bool> attr[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!attr[dev & 63]) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(kSmemBudget));
+  if (!attr[dev & 63].load(std::memory_order_acquire)) {
+    const cudaError_t e = set_smem_attrs(kern, static_cast<int>(kSmemBudget));
     if (e != cudaSuccess) return e;
-    attr[dev & 63] = true;
+    attr[dev & 63].store(true, std::memory_order_release);
   }
   const int grid = ntiles < sms ? ntiles : sms;
   const uint64_t tile_bytes = static_cast<uint64_t>(kTR) * (a.K / 2 + 4 * G);
@@ -409,7 +623,14 @@ cudaError_t launch_tma_m(const GemvArgs& a, int sms, cudaStream_t st) {
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, *map, a.X, a.ldx, a.S, a.Z, a.N, a.K, c.NS, c.CG,
-                            prefetch_tiles, a.Y, a.ldy, a.status);
+                            c.x_staged ? 1 : 0, c.sz_slots, prefetch_tiles, a.Y, a.ldy,
+                            a.status);
+}
+
+template <int M>
+cudaError_t launch_tma_m(const GemvArgs& a, int sms, cudaStream_t st) {
+  if (M == 1 && a.K / 128 <= kIntMaxG) return launch_tma_k<M, true>(a, sms, st);
+  return launch_tma_k<M, false>(a, sms, st);
 }
 
 }  // namespace
@@ -418,7 +639,8 @@ bool gemv_tma_ok(const GemvArgs& a) {
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   return a.M >= 1 && a.M <= 4 && a.K % 128 == 0 && a.group == 128 && a.sz_row == a.K / 128 &&
          a.N % kTR == 0 && (a.ldx % 8) == 0 && al16(a.X) && al16(a.P) && al16(a.S) &&
-         al16(a.Z) && tma_config(a.M, a.K / 128).NS > 0;
+         al16(a.Z) &&
+         tma_config(a.M, a.K / 128, a.M == 1 && a.K / 128 <= kIntMaxG).NS > 0;
 }
 
 cudaError_t launch_gemv_tma(const GemvArgs& a, int sms, cudaStream_t st) {

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <initializer_list>
 #include <stdint.h>
 
 namespace wq {
@@ -10,6 +11,8 @@ namespace wq {
 // SM count and device address of the status word for the current device (false if there
 // is no usable sm_100 device). Defined in api.cu.
 bool current_device(int* sms, unsigned** status);
+// Every non-null pointer is memory of the current device (or managed memory). api.cu.
+bool pointers_on_current_device(std::initializer_list<const void*> ptrs);
 
 // sym: symmetric INT4 (s' = max|w|/7, Z = 8) in the same storage.
 cudaError_t launch_quant_asym(const void* W, bool bf16, int64_t ldw, int N, int K, int group,
@@ -45,6 +48,10 @@ int gemv_max_k();
 // Streaming TMA-fed decode kernel for M <= 4, g = 128 (decode.cu).
 bool gemv_stream_ok(const GemvArgs& a);
 bool gemv_stream_fits(const GemvArgs& a);
+// Integer-MMA decode kernel for M <= 2, g = 128, short rows: whole-row tiles by bulk copies
+// (gemv_imma.cu).
+bool gemv_imma_bulk_ok(const GemvArgs& a);
+cudaError_t launch_gemv_imma_bulk(const GemvArgs& a, int sms, cudaStream_t st);
 // 32-row-tile TMA-fed decode kernel for M <= 4, g = 128, N % 32 == 0 (gemv_tma.cu).
 bool gemv_tma_ok(const GemvArgs& a);
 cudaError_t launch_gemv_tma(const GemvArgs& a, int sms, cudaStream_t st);

@@ -28,28 +28,27 @@ static __device__ __align__(256) float2 g_noalloc_ranges[kNoAllocMaxRanges];
 
 constexpr int kMaxDevices = 64;
 struct NoAllocDevice {
-  bool ready = false;
-  bool ok = false;
-  float2* ranges = nullptr;  // device address of g_noalloc_ranges on this device
+  float2* ranges = nullptr;  // device address of g_noalloc_ranges on this device, once known
 };
 NoAllocDevice g_na[kMaxDevices];
 std::mutex g_na_mu;
 
-// Device address of the scratch array on the current device (nullptr on failure).
+// Device address of the scratch array on the current device (nullptr on failure). Only a
+// successful lookup is kept, so a failed one (for example inside a stream capture) is
+// retried by the next call instead of failing every later call on that device.
 float2* scratch_address() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_na_mu);
   NoAllocDevice& d = g_na[dev];
-  if (!d.ready) {
-    d.ready = true;
+  if (!d.ranges) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_ranges) == cudaSuccess && p != nullptr) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_ranges) == cudaSuccess && p != nullptr)
       d.ranges = static_cast<float2*>(p);
-      d.ok = true;
-    }
+    else
+      cudaGetLastError();  // clear the error of the failed lookup
   }
-  return d.ok ? d.ranges : nullptr;
+  return d.ranges;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -72,6 +71,7 @@ extern "C" wq_status wq_quantize_rtn_per_tensor_noalloc(const void* W, wq_dtype 
   int sms = 0;
   unsigned* status = nullptr;
   if (!wq::current_device(&sms, &status)) return WQ_ERR_NODEVICE;
+  if (!wq::pointers_on_current_device({W, packed, S, Z})) return WQ_ERR_DEVICE;
   // The range pass uses one (min, max) slot per CTA, 8 CTAs per SM.
   const int nparts = wq::per_tensor_parts(sms);
   if (nparts > kNoAllocMaxRanges) return WQ_ERR_UNSUPPORTED;

@@ -163,6 +163,13 @@ __device__ __forceinline__ void tma_prefetch_3d(const void* map, int x, int y, i
                : "memory");
 }
 
+// Hint: bring the box at (x, y) of a 2D tensor map into L2 (safe before pdl_wait()).
+__device__ __forceinline__ void tma_prefetch_2d(const void* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // Bring a tensor map (a __grid_constant__ kernel parameter) into the TMA unit's cache.
 __device__ __forceinline__ void prefetch_tensormap(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");

@@ -20,7 +20,10 @@
 //               quarter), round to bf16, stage [256 tokens x 128 rows] in shared memory
 //               and write it to Y with one TMA store per tile.
 // Every mbarrier wait is bounded (2 s): on a timeout the kernel records kStTimeout and all
-// roles leave their loops, drain outstanding work with bounded waits, free TMEM and exit.
+// roles leave their loops; the TMA lane waits (bounded) for the copies it issued, the MMA
+// lane for its last commit, and the CTA frees TMEM and exits.
+#include <atomic>
+
 #include "common.cuh"
 #include "ptx.cuh"
 #include "tc_gemm.h"
@@ -262,6 +265,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         }
         if (!ok) break;
       }
+      // never leave with copies in flight (also after an abort): wait, bounded, for the last
+      // fill of every stage this lane issued
+      for (uint32_t s = 0; s < static_cast<uint32_t>(kStages) && s < it; ++s) {
+        const uint32_t last = (it - 1 - s) / kStages;
+        if (!mbar_wait_bounded(&sm->raw_full[s], last & 1u, kLimitNs)) set_status(status, kStTimeout);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer
@@ -451,12 +460,14 @@ wq_status launch_tc_gemm(const TcGemmArgs& a, int sms, unsigned* status, cudaStr
   }
   auto kern = int8 ? tc_gemm_kernel<true> : tc_gemm_kernel<false>;
   const size_t smem = int8 ? smem_bytes<true>() : smem_bytes<false>();
-  static bool attr[2] = {false, false};
-  if (!attr[int8]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+  // the attribute is per device: set it on each device's first call (flags by device)
+  static std::atomic<bool> attr[64][2];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
+  if (!attr[dev & 63][int8].load(std::memory_order_acquire)) {
+    if (set_smem_attrs(kern, static_cast<int>(smem)) != cudaSuccess)
       return WQ_ERR_CUDA;
-    attr[int8] = true;
+    attr[dev & 63][int8].store(true, std::memory_order_release);
   }
   const int tiles = ((a.N + kRows - 1) / kRows) * ((a.M + kToks - 1) / kToks);
   const int grid = tiles < sms ? tiles : sms;
