@@ -20,6 +20,15 @@ Sources (page title, section):
         section "The vocabulary": W4A16 dequantizes 4-bit weights to 16 bits inside the
         kernel and runs a 16-bit matmul, Y = X W^T; section "Granularity and outliers":
         the symmetric quantize-dequantize demo and its relative Frobenius errors.
+  [SQ]  same page, "Granularity and outliers": SmoothQuant's per-input-channel factor
+        s_j = max|X_j|^alpha / max|W_j|^(1 - alpha) (alpha = 0.5), with X/s and W*s
+        giving the same product X W^T.
+  [AW]  same page, "GPTQ vs AWQ: two ways to choose what error to keep": AWQ scales the
+        weight columns of large-activation channels up by s (activations down by s)
+        before rounding; s = mean|X_j|^a normalised so that sqrt(max s * min s) = 1, the
+        exponent a chosen on calibration data by the output error. Also "DL S067 -
+        Quantization", section 5 "AWQ intuition" (y = (W diag(s)) (diag(1/s) x), 1/s
+        pushed into the previous layer), and "Model Quantization", section 2.2.
 
 Readings where the pages are silent (each is pinned by a test in tests/test_oracle.py):
   * range includes zero: alpha = min(0, min w), beta = max(0, max w);
@@ -34,7 +43,16 @@ Readings where the pages are silent (each is pinned by a test in tests/test_orac
   * symmetric INT4 per group [GR]: s = max|w|/7 rounded once to binary16 (0 -> 1.0),
     q = clip(RNE(w/s'), -8, 7) on the exact quotient, stored as q + 8 with Z = 8;
   * a matmul "on the same dequantized weights" uses either the exact S'(q - Z)
-    ("exact" mode) or its bfloat16 rounding ("bf16" mode).
+    ("exact" mode) or its bfloat16 rounding ("bf16" mode);
+  * scale folding [SQ][AW]: the folded weight W*s is rounded once to float32 (the
+    precision in which a kernel forms it) before the RTN steps above; the folded
+    activation X/s is the float32 quotient rounded to bfloat16 (the activations' storage
+    type); every s_j must be finite and > 0;
+  * a channel whose statistic is zero (max|X_j| or max|W_j| for SmoothQuant, mean|X_j|
+    for AWQ) gets s_j = 1 and is left out of AWQ's normalisation (the pages' formulas
+    give 0/0 or 0 there);
+  * the per-channel mean |X_j| is the column's exact sum (math.fsum, exact whenever the
+    sum fits binary64's 53 bits) divided by the row count and rounded once to float32.
 
 Parity status: every function below is pinned by tests/test_oracle.py. The pages print
 no values for the outlier-stress construction, so ``outlier_quality`` is pinned by
@@ -57,7 +75,9 @@ __all__ = [
     "Q4S_MIN", "Q4S_MAX", "quantize_rtn_sym_int4", "sym_int4_storage",
     "matmul_f64", "w4a16_matmul", "w8a16_matmul", "qdq_sym", "rel_frobenius",
     "gemm_gate", "bits_per_weight", "decode_ceiling_tok_s", "error_bound_ok",
-    "outlier_quality",
+    "outlier_quality", "f32_round", "channel_absmax", "channel_absmean", "smooth_scales",
+    "smoothquant_scales", "awq_scales", "fold_input_scales", "fold_weight_f32",
+    "quantize_rtn_scaled", "scale_activations_bf16", "awq_search",
 ]
 
 Q4_MIN, Q4_MAX = 0, 15       # asymmetric INT4 integer range [CM]
@@ -89,6 +109,25 @@ def fp16_round(r) -> float:
     n = round(a / ulp)              # Python rounds a Fraction half to even
     v = n * ulp
     if v > FP16_MAX:
+        return sign * math.inf
+    return sign * float(v)
+
+
+def f32_round(r) -> float:
+    """Round an exact rational (or float) to the nearest binary32 value, ties to even
+    (subnormals included); +-inf on overflow. Returned as an exact Python float."""
+    r = Fraction(r)
+    if r == 0:
+        return 0.0
+    sign = -1.0 if r < 0 else 1.0
+    a = abs(r)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if a < Fraction(2) ** e:
+        e -= 1                      # 2**e <= a < 2**(e+1)
+    e = max(e, -126)                # subnormal spacing 2**-149
+    ulp = Fraction(2) ** (e - 23)   # 23 fraction bits
+    v = round(a / ulp) * ulp
+    if v > Fraction(float(np.finfo(np.float32).max)):
         return sign * math.inf
     return sign * float(v)
 
@@ -365,3 +404,116 @@ def outlier_quality(W, X, group):
     W_hat = dequant_asym(codes, S, Z, group)
     W64 = np.asarray(W, dtype=np.float64)
     return rel_frobenius(W64, W_hat), rel_frobenius(matmul_f64(X, W64), matmul_f64(X, W_hat))
+
+
+# ------------------------------------------------ per-input-channel scale folding [SQ][AW]
+
+def channel_absmax(A) -> np.ndarray:
+    """max_i |A_ij| for every column j of A [rows, cols] (exact)."""
+    return np.abs(np.asarray(A, dtype=np.float64)).max(axis=0)
+
+
+def channel_absmean(A) -> np.ndarray:
+    """mean_i |A_ij| per column j, rounded once to float32 (returned as float64):
+    the column sum by math.fsum (correctly rounded, so exact when it fits 53 bits),
+    then the exact quotient by the row count rounded to float32."""
+    A = np.abs(np.asarray(A, dtype=np.float64))
+    rows = A.shape[0]
+    return np.array([f32_round(Fraction(math.fsum(A[:, j])) / rows)
+                     for j in range(A.shape[1])])
+
+
+def smooth_scales(xmax, wmax, alpha=0.5) -> np.ndarray:
+    """SmoothQuant migration factors [SQ] from per-channel statistics:
+    s_j = xmax_j^alpha / wmax_j^(1 - alpha); s_j = 1 where either statistic is zero."""
+    xmax = np.asarray(xmax, dtype=np.float64)
+    wmax = np.asarray(wmax, dtype=np.float64)
+    s = np.ones_like(xmax)
+    live = (xmax > 0) & (wmax > 0)
+    s[live] = xmax[live] ** alpha / wmax[live] ** (1.0 - alpha)
+    return s
+
+
+def smoothquant_scales(X, W, alpha=0.5) -> np.ndarray:
+    """s for activations X [tokens, K] and weights W [out, K]: the column maxima of |X|
+    (over tokens) and of |W| (over output rows) fed to ``smooth_scales`` [SQ]."""
+    return smooth_scales(channel_absmax(X), channel_absmax(W), alpha)
+
+
+def awq_scales(a_mag, alpha) -> np.ndarray:
+    """AWQ factors [AW]: s_j = a_j^alpha divided by sqrt(max_j s_j * min_j s_j), so that
+    the factors are centred on 1 in log scale; a channel with a_j = 0 gets s_j = 1 and is
+    left out of the max and min."""
+    a = np.asarray(a_mag, dtype=np.float64)
+    s = np.ones_like(a)
+    live = a > 0
+    if np.any(live):
+        p = a[live] ** alpha
+        s[live] = p / math.sqrt(float(p.max()) * float(p.min()))
+    return s
+
+
+def _check_factors(s):
+    s = np.asarray(s, dtype=np.float64)
+    if not np.all(np.isfinite(s)) or np.any(s <= 0):
+        raise ValueError("scale factors must be finite and positive")
+    return s
+
+
+def fold_input_scales(X, W, s):
+    """(X / s, W * s) in float64 [SQ][AW]: activations divided and weight columns
+    multiplied by the same per-input-channel factor, so (X/s)(W s)^T = X W^T."""
+    s = _check_factors(s)
+    return np.asarray(X, dtype=np.float64) / s, np.asarray(W, dtype=np.float64) * s
+
+
+def fold_weight_f32(W, s) -> np.ndarray:
+    """W * s per input channel, rounded once to float32 (returned as float64). W and s
+    hold float32 values, whose product (at most 48 significant bits) float64 holds
+    exactly, so the cast below is the only rounding."""
+    s = _check_factors(s)
+    P = np.asarray(W, dtype=np.float64) * s
+    with np.errstate(over="ignore"):
+        P32 = P.astype(np.float32)
+    if not np.all(np.isfinite(P32)):
+        raise NonFiniteError("folded weight is not finite in float32")
+    return P32.astype(np.float64)
+
+
+def quantize_rtn_scaled(W, s, group=128, sym=False):
+    """RTN INT4 of the folded weight W * s (``fold_weight_f32``) [AW]: asymmetric (codes,
+    S, Z) as ``quantize_rtn_asym``, or symmetric in the stored form of
+    ``sym_int4_storage``."""
+    Wf = fold_weight_f32(W, s)
+    if sym:
+        return sym_int4_storage(*quantize_rtn_sym_int4(Wf, group))
+    return quantize_rtn_asym(Wf, group)
+
+
+def scale_activations_bf16(X, s) -> np.ndarray:
+    """bfloat16 bits of X / s [SQ][AW]: the float32 quotient (float64 division of two
+    float32 values rounded to float32 equals the correctly rounded float32 quotient,
+    since 53 >= 2*24 + 2), then rounded to bfloat16, ties to even."""
+    s = _check_factors(s)
+    q = (np.asarray(X, dtype=np.float64) / s).astype(np.float32)
+    return bf16_round_bits(q)
+
+
+def awq_search(W, X, alphas, qdq):
+    """AWQ's exponent search [AW]: a_j = mean_i |X_ij| on the calibration set X; for each
+    candidate exponent a (in the given order) fold s = ``awq_scales``(a_mag, a) into the
+    weight columns, quantize-dequantize with ``qdq``, fold 1/s back, and score
+    ||X W^T - X Q^T||_F. Returns (Q, a, s) of the first candidate with the smallest
+    score."""
+    W = np.asarray(W, dtype=np.float64)
+    X = np.asarray(X, dtype=np.float64)
+    a_mag = np.abs(X).mean(axis=0)
+    Y = X @ W.T
+    best = None
+    for a in alphas:
+        s = awq_scales(a_mag, a)
+        Q = qdq(W * s) / s
+        err = np.linalg.norm(Y - X @ Q.T)
+        if best is None or err < best[0]:
+            best = (err, a, Q, s)
+    return best[2], best[1], best[3]

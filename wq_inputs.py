@@ -105,3 +105,28 @@ def granularity_demo_tensors():
     ch = rng.choice(1024, 6, replace=False)
     X[:, ch] *= 50
     return W, X
+
+
+def calibration_toy_tensors():
+    """The calibration toy on the study-docs page ("LLM Weight Quantization ...",
+    section "GPTQ vs AWQ: two ways to choose what error to keep"), drawn in the same
+    order from ``default_rng(1)``: a d x d mixing matrix N(0,1)/sqrt(d) (d = 128), 4
+    distinct "salient" channels whose activations are 8x larger, a calibration set and a
+    held-out set of 1024 correlated activations each (standard normals times the mixing
+    matrix, plus 0.3 times independent standard normals, times the channel factors), and
+    W 64x128 ~N(0, 0.05). Returns (W, X_cal, X_test), float64. The mixing only shapes the
+    synthetic activations; no quantization arithmetic happens here."""
+    rng = np.random.default_rng(1)
+    d, rows, n = 128, 64, 1024
+    mix = rng.normal(0, 1, (d, d)) / np.sqrt(d)
+    chan = np.ones(d)
+    chan[rng.choice(d, 4, replace=False)] = 8.0
+
+    def draw(m):
+        base = rng.normal(0, 1, (m, d)) @ mix
+        return (base + 0.3 * rng.normal(0, 1, (m, d))) * chan
+
+    X_cal = draw(n)
+    X_test = draw(n)
+    W = rng.normal(0, 0.05, (rows, d))
+    return W, X_cal, X_test
