@@ -59,14 +59,17 @@ extern "C" {
 typedef enum wq_status {
   WQ_OK = 0,
   WQ_ERR_NULL = 1,        /* a required pointer is NULL                          */
-  WQ_ERR_SHAPE = 2,       /* sizes <= 0, K % g != 0, K odd, ld too small, ...    */
+  WQ_ERR_SHAPE = 2,       /* sizes <= 0, K % g != 0, ld too small, alpha outside  */
+                          /* [0, 1], ...                                          */
   WQ_ERR_ALIGN = 3,       /* a pointer or leading dimension breaks 16-B alignment */
   WQ_ERR_DTYPE = 4,       /* dtype not supported by this call                    */
   WQ_ERR_UNSUPPORTED = 5, /* parameter combination not implemented               */
   WQ_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed                */
   WQ_ERR_NONFINITE = 7,   /* device: NaN/inf weight or binary16 scale overflow   */
   WQ_ERR_TIMEOUT = 8,     /* device: a bounded barrier wait gave up              */
-  WQ_ERR_RANGE = 9,       /* device: a code given to wq_pack_int4 exceeds 15     */
+  WQ_ERR_RANGE = 9,       /* device: a code given to wq_pack_int4 exceeds 15, or */
+                          /* a factor s_j given to wq_quantize_rtn_scaled is not */
+                          /* finite and > 0                                       */
   WQ_ERR_NODEVICE = 10,   /* no CUDA device, or it is not sm_100                 */
   WQ_ERR_DEVICE = 11      /* a pointer is not memory of the current device      */
 } wq_status;
@@ -171,6 +174,58 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
 wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t* codes,
                         const uint16_t* S, int64_t N, int64_t K, uint16_t* Y, int64_t ldy,
                         void* stream);
+
+/* ---- Per-input-channel scale folding ("LLM Weight Quantization ...", sections
+ * "Granularity and outliers" (SmoothQuant) and "GPTQ vs AWQ: two ways to choose what error
+ * to keep" (AWQ); "DL S067 - Quantization", section 5 "AWQ intuition"). A factor s_j > 0
+ * per input channel j multiplies weight column j before round-to-nearest and divides
+ * activation column j, so that (X / s)(W diag(s))^T = X W^T. At serve time the folded
+ * codes run on wq_w4a16_gemm unchanged, with activations X / s: either produced by the
+ * previous layer (1/s folded into its weights, as the AWQ section suggests) or by
+ * wq_scale_activations below. s is float32 [K], device memory. */
+
+/* Per-column statistic of A [rows, cols] (fp32 or bf16, row stride lda elements):
+ *   WQ_STAT_ABSMAX   out[j] = max_i |A_ij| (exact; a NaN propagates);
+ *   WQ_STAT_ABSMEAN  out[j] = mean_i |A_ij|: float64 sums, the quotient by rows rounded once
+ *                    to float32 (exact whenever the column's sum fits 53 bits).
+ * The factor formulas below take these: max |X_j| over calibration tokens and max |W_j|
+ * over output rows (SmoothQuant), mean |X_j| (AWQ). The result is deterministic.
+ * Requires rows >= 1 (else WQ_ERR_SHAPE; cols == 0 is a no-op), cols % 8 == 0, lda >= cols,
+ * A and lda * element size 16-byte aligned, out [cols] float32. */
+typedef enum wq_stat { WQ_STAT_ABSMAX = 0, WQ_STAT_ABSMEAN = 1 } wq_stat;
+wq_status wq_channel_stat(const void* A, wq_dtype dtype, int64_t rows, int64_t cols,
+                          int64_t lda, int32_t stat, float* out, void* stream);
+
+/* SmoothQuant factors s_j = xmax_j^alpha / wmax_j^(1 - alpha) ("Granularity and outliers";
+ * alpha = 0.5 there), computed in float64 and rounded to float32; s_j = 1 where xmax_j or
+ * wmax_j is not > 0. xmax, wmax, s: float32 [K]. alpha in [0, 1], else WQ_ERR_SHAPE. */
+wq_status wq_smooth_scales(const float* xmax, const float* wmax, int64_t K, float alpha,
+                           float* s, void* stream);
+
+/* AWQ factors for one exponent alpha ("GPTQ vs AWQ ..."): p_j = a_j^alpha over the channels
+ * with a_j > 0 (a = mean |X_j| on calibration data), s_j = p_j / sqrt(max p * min p) so that
+ * the factors are centred on 1; s_j = 1 where a_j is not > 0. float64 arithmetic, float32
+ * result. alpha in [0, 1], else WQ_ERR_SHAPE. One CTA (K is one layer's input width). */
+wq_status wq_awq_scales(const float* a_mag, int64_t K, float alpha, float* s, void* stream);
+
+/* Round-to-nearest INT4 of the folded weights W diag(s): w'_nk = w_nk * s_k rounded once to
+ * float32, then exactly the steps and outputs of wq_quantize_rtn_g128 for {4, g, 1} or
+ * {4, g, 0} (params NULL = {4, 128, 1}; g a multiple of 32 dividing K). A factor that is not
+ * finite and > 0 sets WQ_ERR_RANGE in the status word; a folded weight that is not finite,
+ * or a scale overflow, WQ_ERR_NONFINITE. W as for wq_quantize_rtn_g128; s float32 [K],
+ * 16-byte aligned. The dequantized codes approximate W diag(s): multiply by the activations
+ * X / s (or divide the dequantized column by s_k) to approximate W. */
+wq_status wq_quantize_rtn_scaled(const void* W, wq_dtype w_dtype, int64_t N, int64_t K,
+                                 int64_t ldw, const float* s, const wq_qparams* params,
+                                 uint8_t* packed, uint16_t* S, uint16_t* Z, void* stream);
+
+/* Xs = X / s per column: each bf16 x_mk divided by s_k in float32 (round-to-nearest), the
+ * quotient rounded to bfloat16 (ties to even). X, Xs [M, K] bf16 with row strides ldx, ldxs
+ * (multiples of 8, 16-byte aligned bases); s float32 [K], 16-byte aligned; K % 8 == 0.
+ * Xs may be X itself (in place) when ldxs == ldx; other overlaps are undefined. No check of
+ * s: a zero or non-finite factor gives the IEEE quotient. */
+wq_status wq_scale_activations(const uint16_t* X, int64_t M, int64_t K, int64_t ldx,
+                               const float* s, uint16_t* Xs, int64_t ldxs, void* stream);
 
 /* Synchronize `stream`, then return and clear the current device's status word:
  * WQ_OK, or the first of WQ_ERR_NONFINITE / WQ_ERR_RANGE / WQ_ERR_TIMEOUT recorded by a

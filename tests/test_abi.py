@@ -115,6 +115,40 @@ def test_pack_dequant_argument_checks(lib):
     assert p(FAKE, wq.WQ_BF16, 4, 128, 128, FAKE, FAKE, FAKE, None, 0, None) == NULL
 
 
+def test_scale_folding_argument_checks(lib):
+    RANGE_ALPHA = (-0.1, 1.5, float("nan"))
+    c = lib.wq_channel_stat
+    assert c(FAKE, wq.WQ_BF16, 8, 0, 0, 0, FAKE, None) == OK          # no columns: no-op
+    assert c(FAKE, wq.WQ_BF16, 0, 64, 64, 0, FAKE, None) == SHAPE     # statistic over no rows
+    assert c(FAKE, wq.WQ_F16, 8, 64, 64, 0, FAKE, None) == DTYPE
+    assert c(FAKE, wq.WQ_BF16, 8, 64, 64, 2, FAKE, None) == UNSUP     # unknown statistic
+    assert c(None, wq.WQ_BF16, 8, 64, 64, 1, FAKE, None) == NULL
+    assert c(FAKE, wq.WQ_BF16, 8, 60, 64, 0, FAKE, None) == SHAPE     # cols % 8
+    assert c(FAKE, wq.WQ_BF16, 8, 64, 32, 0, FAKE, None) == SHAPE     # lda < cols
+    assert c(ODD, wq.WQ_BF16, 8, 64, 64, 0, FAKE, None) == ALIGN
+    assert c(FAKE, wq.WQ_BF16, 8, 64, 68, 0, FAKE, None) == ALIGN     # row stride 136 B
+    for f, args in ((lib.wq_smooth_scales, lambda a: (FAKE, FAKE, 64, a, FAKE, None)),
+                    (lib.wq_awq_scales, lambda a: (FAKE, 64, a, FAKE, None))):
+        for a in RANGE_ALPHA:
+            assert f(*args(a)) == SHAPE
+    assert lib.wq_smooth_scales(FAKE, None, 64, 0.5, FAKE, None) == NULL
+    assert lib.wq_smooth_scales(FAKE, FAKE, 0, 0.5, None, None) == OK
+    assert lib.wq_awq_scales(None, 64, 0.5, FAKE, None) == NULL
+    q = lib.wq_quantize_rtn_scaled
+    assert q(FAKE, wq.WQ_BF16, 4, 128, 128, None, None, FAKE, FAKE, FAKE, None) == NULL  # no s
+    assert q(FAKE, wq.WQ_BF16, 4, 128, 128, FAKE, _qp(8, 128, 0), FAKE, FAKE, FAKE,
+             None) == UNSUP
+    assert q(FAKE, wq.WQ_BF16, 4, 192, 192, FAKE, None, FAKE, FAKE, FAKE, None) == SHAPE
+    assert q(FAKE, wq.WQ_BF16, 4, 128, 128, ODD, None, FAKE, FAKE, FAKE, None) == ALIGN
+    assert q(FAKE, wq.WQ_I8, 4, 128, 128, FAKE, None, FAKE, FAKE, FAKE, None) == DTYPE
+    a = lib.wq_scale_activations
+    assert a(FAKE, 0, 64, 64, FAKE, FAKE, 64, None) == OK
+    assert a(FAKE, 2, 60, 64, FAKE, FAKE, 64, None) == SHAPE             # K % 8
+    assert a(FAKE, 2, 64, 64, FAKE, FAKE, 32, None) == SHAPE             # ldxs < K
+    assert a(FAKE, 2, 64, 64, ODD, FAKE, 64, None) == ALIGN              # s alignment
+    assert a(FAKE, 2, 64, 64, FAKE, FAKE, 72, None) == UNSUP             # in place, other ld
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="host without a GPU only")
 def test_valid_call_without_device_reports_nodevice(lib):
     """A call that passes every host check but finds no sm_100 device fails loudly

@@ -12,6 +12,11 @@ Functions carry the C names:
     wq_dequant(packed, S, Z, group, out_dtype) -> W_hat
     wq_w4a16_gemm(X, packed, S, Z, group) -> Y
     wq_w8a16_gemm(X, codes, S) -> Y
+    wq_channel_stat(A, stat) -> float32 [cols]      (WQ_STAT_ABSMAX / WQ_STAT_ABSMEAN)
+    wq_smooth_scales(xmax, wmax, alpha) -> s
+    wq_awq_scales(a_mag, alpha) -> s
+    wq_quantize_rtn_scaled(W, s, group=128, zero_point=True) -> (packed, S, Z)
+    wq_scale_activations(X, s) -> X / s
     wq_get_status() -> int
 S and Z are returned as torch.float16 tensors (binary16 bit patterns in the C ABI).
 """
@@ -29,10 +34,13 @@ __all__ = [
     "wq_quantize_per_tensor_workspace_bytes", "wq_quantize_rtn_per_tensor_noalloc",
     "wq_pack_int4", "wq_dequant", "wq_w4a16_gemm",
     "wq_w8a16_gemm", "wq_get_status", "wq_selftest_bounded_wait",
-    "WQ_F32", "WQ_BF16", "WQ_F16", "WQ_U8", "WQ_I8",
+    "wq_channel_stat", "wq_smooth_scales", "wq_awq_scales", "wq_quantize_rtn_scaled",
+    "wq_scale_activations",
+    "WQ_F32", "WQ_BF16", "WQ_F16", "WQ_U8", "WQ_I8", "WQ_STAT_ABSMAX", "WQ_STAT_ABSMEAN",
 ]
 
 WQ_F32, WQ_BF16, WQ_F16, WQ_U8, WQ_I8 = 0, 1, 2, 3, 4
+WQ_STAT_ABSMAX, WQ_STAT_ABSMEAN = 0, 1
 STATUS_NAMES = {
     0: "WQ_OK", 1: "WQ_ERR_NULL", 2: "WQ_ERR_SHAPE", 3: "WQ_ERR_ALIGN", 4: "WQ_ERR_DTYPE",
     5: "WQ_ERR_UNSUPPORTED", 6: "WQ_ERR_CUDA", 7: "WQ_ERR_NONFINITE", 8: "WQ_ERR_TIMEOUT",
@@ -70,6 +78,12 @@ _SIGNATURES = {
     "wq_w4a16_gemm": (_I32, [_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I32, _P, _I64, _P]),
     "wq_w8a16_gemm": (_I32, [_P, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _P]),
     "wq_get_status": (_I32, [_P]),
+    "wq_channel_stat": (_I32, [_P, _I32, _I64, _I64, _I64, _I32, _P, _P]),
+    "wq_smooth_scales": (_I32, [_P, _P, _I64, ctypes.c_float, _P, _P]),
+    "wq_awq_scales": (_I32, [_P, _I64, ctypes.c_float, _P, _P]),
+    "wq_quantize_rtn_scaled": (_I32, [_P, _I32, _I64, _I64, _I64, _P, ctypes.POINTER(_QParams),
+                                      _P, _P, _P, _P]),
+    "wq_scale_activations": (_I32, [_P, _I64, _I64, _I64, _P, _P, _I64, _P]),
     "wq_selftest_bounded_wait": (_I32, [ctypes.c_uint64, _I32, _P]),
 }
 
@@ -325,6 +339,84 @@ def wq_w8a16_gemm(X, codes, S, Y=None, stream=None):
                                  _stream(stream))
     _check(st, "wq_w8a16_gemm")
     return Y
+
+
+def wq_channel_stat(A, stat: int = WQ_STAT_ABSMAX, out=None, stream=None):
+    """Per-column max |A_ij| (WQ_STAT_ABSMAX) or mean |A_ij| (WQ_STAT_ABSMEAN) of A [rows,
+    cols] (float32 or bfloat16) -> float32 [cols]."""
+    import torch
+
+    rows, cols = A.shape
+    lda = _rows(A, "A")
+    out = torch.empty((cols,), dtype=torch.float32, device=A.device) if out is None else out
+    with _on_device(A):
+        st = lib().wq_channel_stat(_ptr(A), _w_dtype(A), rows, cols, lda, int(stat), _ptr(out),
+                                   _stream(stream))
+    _check(st, "wq_channel_stat")
+    return out
+
+
+def wq_smooth_scales(xmax, wmax, alpha: float = 0.5, out=None, stream=None):
+    """SmoothQuant factors s_j = xmax_j^alpha / wmax_j^(1 - alpha), float32 [K]."""
+    import torch
+
+    K = xmax.shape[0]
+    out = torch.empty((K,), dtype=torch.float32, device=xmax.device) if out is None else out
+    with _on_device(xmax):
+        st = lib().wq_smooth_scales(_ptr(xmax), _ptr(wmax), K, float(alpha), _ptr(out),
+                                    _stream(stream))
+    _check(st, "wq_smooth_scales")
+    return out
+
+
+def wq_awq_scales(a_mag, alpha: float, out=None, stream=None):
+    """AWQ factors a_j^alpha / sqrt(max * min), float32 [K]."""
+    import torch
+
+    K = a_mag.shape[0]
+    out = torch.empty((K,), dtype=torch.float32, device=a_mag.device) if out is None else out
+    with _on_device(a_mag):
+        st = lib().wq_awq_scales(_ptr(a_mag), K, float(alpha), _ptr(out), _stream(stream))
+    _check(st, "wq_awq_scales")
+    return out
+
+
+def wq_quantize_rtn_scaled(W, s, group: int = 128, zero_point: bool = True, packed=None,
+                           S=None, Z=None, stream=None):
+    """RTN INT4 of W diag(s) (W [N, K] float32 or bfloat16, s float32 [K]): returns
+    (packed uint8 [N, K/2], S fp16 [N, K/g], Z fp16 [N, K/g]) as wq_quantize_rtn_g128."""
+    import torch
+
+    N, K = W.shape
+    ldw = _rows(W, "W")
+    dev = W.device
+    G = K // group if group else 1
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev) if packed is None else packed
+    S = torch.empty((N, G), dtype=torch.float16, device=dev) if S is None else S
+    Z = torch.empty((N, G), dtype=torch.float16, device=dev) if Z is None else Z
+    p = _QParams(4, group, 1 if zero_point else 0)
+    with _on_device(W):
+        st = lib().wq_quantize_rtn_scaled(_ptr(W), _w_dtype(W), N, K, ldw, _ptr(s),
+                                          ctypes.byref(p), _ptr(packed), _ptr(S), _ptr(Z),
+                                          _stream(stream))
+    _check(st, "wq_quantize_rtn_scaled")
+    return packed, S, Z
+
+
+def wq_scale_activations(X, s, out=None, stream=None):
+    """X / s per column (X [M, K] bfloat16, s float32 [K]) -> bfloat16 [M, K]; out may be
+    X itself."""
+    import torch
+
+    M, K = X.shape
+    ldx = _rows(X, "X")
+    out = torch.empty((M, K), dtype=torch.bfloat16, device=X.device) if out is None else out
+    ldo = _rows(out, "out")
+    with _on_device(X):
+        st = lib().wq_scale_activations(_ptr(X), M, K, ldx, _ptr(s), _ptr(out), ldo,
+                                        _stream(stream))
+    _check(st, "wq_scale_activations")
+    return out
 
 
 def wq_selftest_bounded_wait(limit_ns: int = 20_000_000, spin: bool = True, stream=None) -> None:

@@ -99,14 +99,14 @@ const char* wq_status_string(wq_status s) {
   switch (s) {
     case WQ_OK: return "ok";
     case WQ_ERR_NULL: return "a required pointer is NULL";
-    case WQ_ERR_SHAPE: return "invalid sizes (N, K, M, group or leading dimension)";
+    case WQ_ERR_SHAPE: return "invalid sizes (N, K, M, group, leading dimension) or alpha";
     case WQ_ERR_ALIGN: return "pointer or leading dimension not 16-byte aligned";
     case WQ_ERR_DTYPE: return "dtype not supported by this call";
     case WQ_ERR_UNSUPPORTED: return "parameter combination not supported";
     case WQ_ERR_CUDA: return "CUDA runtime error";
     case WQ_ERR_NONFINITE: return "non-finite weight or scale overflow";
     case WQ_ERR_TIMEOUT: return "device wait timed out";
-    case WQ_ERR_RANGE: return "code out of range [0, 15]";
+    case WQ_ERR_RANGE: return "code above 15, or a scale factor not finite and positive";
     case WQ_ERR_NODEVICE: return "no usable sm_100 CUDA device";
     case WQ_ERR_DEVICE: return "a pointer is not memory of the current device";
   }
@@ -282,6 +282,94 @@ wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t*
   }
   wq::TcGemmArgs a{X, ldx, nullptr, S, nullptr, codes, (int)M, (int)N, (int)K, (int)K, 1, Y, ldy};
   return wq::launch_tc_gemm(a, d->sms, d->status, st);
+}
+
+wq_status wq_channel_stat(const void* A, wq_dtype dtype, int64_t rows, int64_t cols,
+                          int64_t lda, int32_t stat, float* out, void* stream) {
+  if (rows < 0 || cols < 0) return WQ_ERR_SHAPE;
+  if (dtype != WQ_F32 && dtype != WQ_BF16) return WQ_ERR_DTYPE;
+  if (stat != WQ_STAT_ABSMAX && stat != WQ_STAT_ABSMEAN) return WQ_ERR_UNSUPPORTED;
+  if (cols == 0) return WQ_OK;
+  if (rows == 0) return WQ_ERR_SHAPE;  // a statistic over no rows
+  if (!A || !out) return WQ_ERR_NULL;
+  if (!fits_int(cols) || cols % 8 != 0 || lda < cols) return WQ_ERR_SHAPE;
+  const size_t es = dtype == WQ_F32 ? 4 : 2;
+  if (!aligned(A, 16) || (lda * es) % 16 != 0 || !aligned(out, 4)) return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({A, out})) return WQ_ERR_DEVICE;
+  return from_cuda(wq::launch_channel_stat(A, dtype == WQ_BF16, lda, rows, (int)cols,
+                                           stat == WQ_STAT_ABSMEAN, out, d->sms,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+// alpha in [0, 1] (the migration strength / the AWQ exponent).
+static bool alpha_ok(float alpha) { return alpha >= 0.0f && alpha <= 1.0f; }
+
+wq_status wq_smooth_scales(const float* xmax, const float* wmax, int64_t K, float alpha,
+                           float* s, void* stream) {
+  if (K < 0 || !alpha_ok(alpha)) return WQ_ERR_SHAPE;
+  if (K == 0) return WQ_OK;
+  if (!xmax || !wmax || !s) return WQ_ERR_NULL;
+  if (!fits_int(K)) return WQ_ERR_SHAPE;
+  if (!aligned(xmax, 4) || !aligned(wmax, 4) || !aligned(s, 4)) return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({xmax, wmax, s})) return WQ_ERR_DEVICE;
+  return from_cuda(wq::launch_smooth_scales(xmax, wmax, (int)K, alpha, s, d->sms,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_awq_scales(const float* a_mag, int64_t K, float alpha, float* s, void* stream) {
+  if (K < 0 || !alpha_ok(alpha)) return WQ_ERR_SHAPE;
+  if (K == 0) return WQ_OK;
+  if (!a_mag || !s) return WQ_ERR_NULL;
+  if (!fits_int(K)) return WQ_ERR_SHAPE;
+  if (!aligned(a_mag, 4) || !aligned(s, 4)) return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({a_mag, s})) return WQ_ERR_DEVICE;
+  return from_cuda(wq::launch_awq_scales(a_mag, (int)K, alpha, s,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_quantize_rtn_scaled(const void* W, wq_dtype w_dtype, int64_t N, int64_t K,
+                                 int64_t ldw, const float* s, const wq_qparams* params,
+                                 uint8_t* packed, uint16_t* S, uint16_t* Z, void* stream) {
+  const wq_qparams p = params ? *params : wq_qparams{4, 128, 1};
+  if (N < 0 || K < 0) return WQ_ERR_SHAPE;
+  if (w_dtype != WQ_F32 && w_dtype != WQ_BF16) return WQ_ERR_DTYPE;
+  if (p.w_bit != 4 || (p.zero_point != 0 && p.zero_point != 1)) return WQ_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return WQ_OK;
+  if (!W || !s || !packed || !S || !Z) return WQ_ERR_NULL;
+  if (!fits_int(N) || !fits_int(K) || K % 32 != 0 || ldw < K) return WQ_ERR_SHAPE;
+  if (p.group < 32 || p.group % 32 != 0 || K % p.group != 0) return WQ_ERR_SHAPE;
+  const size_t es = w_dtype == WQ_F32 ? 4 : 2;
+  if (!aligned(W, 16) || (ldw * es) % 16 != 0 || !aligned(s, 16) || !aligned(packed, 16) ||
+      !aligned(S, 2) || !aligned(Z, 2))
+    return WQ_ERR_ALIGN;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({W, s, packed, S, Z})) return WQ_ERR_DEVICE;
+  return from_cuda(wq::launch_quant_scaled(W, w_dtype == WQ_BF16, ldw, (int)N, (int)K, p.group,
+                                           s, packed, S, Z, p.zero_point == 0, d->status,
+                                           d->sms, static_cast<cudaStream_t>(stream)));
+}
+
+wq_status wq_scale_activations(const uint16_t* X, int64_t M, int64_t K, int64_t ldx,
+                               const float* s, uint16_t* Xs, int64_t ldxs, void* stream) {
+  if (M < 0 || K < 0) return WQ_ERR_SHAPE;
+  if (M == 0 || K == 0) return WQ_OK;
+  if (!X || !s || !Xs) return WQ_ERR_NULL;
+  if (!fits_int(M) || !fits_int(K) || K % 8 != 0 || ldx < K || ldxs < K) return WQ_ERR_SHAPE;
+  if (!aligned(X, 16) || !aligned(Xs, 16) || !aligned(s, 16) || ldx % 8 != 0 || ldxs % 8 != 0)
+    return WQ_ERR_ALIGN;
+  if (X == Xs && ldx != ldxs) return WQ_ERR_UNSUPPORTED;  // in place only row for row
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({X, s, Xs})) return WQ_ERR_DEVICE;
+  return from_cuda(wq::launch_scale_activations(X, ldx, (int)M, (int)K, s, Xs, ldxs, d->sms,
+                                                static_cast<cudaStream_t>(stream)));
 }
 
 wq_status wq_selftest_bounded_wait(uint64_t limit_ns, int32_t spin, void* stream) {

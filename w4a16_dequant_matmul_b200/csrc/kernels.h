@@ -72,6 +72,20 @@ struct Gemv8Args {
 };
 cudaError_t launch_gemv_w8a16(const Gemv8Args& a, cudaStream_t st);
 
+// Per-input-channel scale folding (scale_fold.cu). cols % 8 == 0 for channel_stat.
+cudaError_t launch_channel_stat(const void* A, bool bf16, int64_t lda, int64_t rows, int cols,
+                                bool mean, float* out, int sms, cudaStream_t st);
+cudaError_t launch_smooth_scales(const float* xmax, const float* wmax, int K, float alpha,
+                                 float* s, int sms, cudaStream_t st);
+cudaError_t launch_awq_scales(const float* a_mag, int K, float alpha, float* s,
+                              cudaStream_t st);
+cudaError_t launch_quant_scaled(const void* W, bool bf16, int64_t ldw, int N, int K, int group,
+                                const float* s, uint8_t* packed, uint16_t* S, uint16_t* Z,
+                                bool sym, unsigned* status, int sms, cudaStream_t st);
+cudaError_t launch_scale_activations(const uint16_t* X, int64_t ldx, int M, int K,
+                                     const float* s, uint16_t* Xs, int64_t ldxs, int sms,
+                                     cudaStream_t st);
+
 // One CTA whose single bounded mbarrier wait runs out (selftest.cu).
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, bool spin, unsigned* status,
                                          cudaStream_t st);
