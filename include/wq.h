@@ -211,8 +211,8 @@ wq_status wq_awq_scales(const float* a_mag, int64_t K, float alpha, float* s, vo
 /* Round-to-nearest INT4 of the folded weights W diag(s): w'_nk = w_nk * s_k rounded once to
  * float32, then exactly the steps and outputs of wq_quantize_rtn_g128 for {4, g, 1} or
  * {4, g, 0} (params NULL = {4, 128, 1}; g a multiple of 32 dividing K). A factor that is not
- * finite and > 0 sets WQ_ERR_RANGE in the status word; a folded weight that is not finite,
- * or a scale overflow, WQ_ERR_NONFINITE. W as for wq_quantize_rtn_g128; s float32 [K],
+ * finite and > 0 sets WQ_ERR_RANGE in the status word (its column is folded as 0); a folded
+ * weight that is not finite, or a scale overflow, WQ_ERR_NONFINITE. W as for wq_quantize_rtn_g128; s float32 [K],
  * 16-byte aligned. The dequantized codes approximate W diag(s): multiply by the activations
  * X / s (or divide the dequantized column by s_k) to approximate W. */
 wq_status wq_quantize_rtn_scaled(const void* W, wq_dtype w_dtype, int64_t N, int64_t K,

@@ -342,12 +342,20 @@ def w8a16_matmul(X, codes, s, mode="exact") -> np.ndarray:
     return matmul_f64(X, W_hat)
 
 
-def gemm_gate(y, y_ref) -> float:
-    """max_i |y_i - y_ref_i| / max(|y_ref_i|, 1e-3 * rms(y_ref)): relative error with a
-    floor, so that outputs that cross zero do not make the ratio unbounded."""
+def gemm_gate(y, y_ref, K=None) -> float:
+    """max_i |y_i - y_ref_i| / max(|y_ref_i|, floor): relative error with a floor, so that
+    outputs that cross zero do not make the ratio unbounded.
+
+    floor = 1e-3 * rms(y_ref), or, given the contraction length K, at least 100 times the
+    worst-case error of fp32 accumulation in K/16 steps (a tensor core adds one 16-term dot
+    product to its fp32 accumulator per step, losing up to one fp32 ulp, 2^-23 relative, of
+    partial sums of about rms(y_ref) size): floor = max(1e-3, 100 (K/16) 2^-23) rms(y_ref).
+    With the tolerance 1e-2, an output below the floor is then held to that absolute
+    accumulation error rather than to 1 % of itself."""
     y = np.asarray(y, dtype=np.float64)
     y_ref = np.asarray(y_ref, dtype=np.float64)
-    floor = 1e-3 * math.sqrt(float(np.mean(y_ref ** 2))) if y_ref.size else 0.0
+    rel = 1e-3 if K is None else max(1e-3, 100.0 * (K / 16.0) * 2.0 ** -23)
+    floor = rel * math.sqrt(float(np.mean(y_ref ** 2))) if y_ref.size else 0.0
     den = np.maximum(np.abs(y_ref), floor)
     if y.size == 0:
         return 0.0

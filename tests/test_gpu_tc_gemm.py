@@ -86,3 +86,36 @@ def test_tc_gemm_deterministic():
     Y1 = wq.wq_w4a16_gemm(X, packed, S, Z, 128)
     Y2 = wq.wq_w4a16_gemm(X, packed, S, Z, 128)
     assert torch.equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 4096, 11008), (64, 1024, 28672)])
+def test_tc_gemm_long_k_sampled(M, N, K):
+    """Long contractions (the 7B down projection in prefill, a 70B-class K): the tensor core's
+    fp32 accumulation error grows with K, so the gate's floor is the one derived from K."""
+    Wb = wq_inputs.weight_bf16(N, K, 0.015, seed=7)
+    Xb = wq_inputs.act_bf16(M, K, seed=8)
+    packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb))
+    Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, 128)
+    assert wq.wq_get_status() == 0
+    rows = np.sort(np.random.default_rng(6).choice(N, 48, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    codes, So, Zo = oracle.quantize_rtn_asym(wq_inputs.bf16_bits_to_f64(Wb[rows]), 128)
+    np.testing.assert_array_equal(gu.to_np(packed)[rows], oracle.pack_int4(codes))
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "bf16")
+    y = gu.bf16_to_f64(Y)[:, rows]
+    assert oracle.gemm_gate(y, Yref, K) <= GATE
+    assert oracle.rel_frobenius(Yref, y) < 4e-3
+
+
+def test_tc_w8a16_long_k_sampled():
+    M, N, K = 256, 2048, 11008
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=9)
+    Xb = wq_inputs.act_bf16(M, K, seed=10)
+    q, S, _ = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb), 8, K, False)
+    Y = wq.wq_w8a16_gemm(gu.bf16_from_bits(Xb), q, S)
+    assert wq.wq_get_status() == 0
+    rows = np.sort(np.random.default_rng(11).choice(N, 48, replace=False))
+    qo, so = oracle.quantize_sym_int8_per_channel(wq_inputs.bf16_bits_to_f64(Wb[rows]))
+    np.testing.assert_array_equal(gu.to_np(q)[rows], qo)
+    Yref = oracle.w8a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), qo, so, "bf16")
+    assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref, K) <= GATE

@@ -301,6 +301,13 @@ def test_gemm_gate():
     rms = math.sqrt(np.mean(ref ** 2))
     assert math.isclose(oracle.gemm_gate(ref + [0, 0, 1e-3, 0], ref), 1e-3 / (1e-3 * rms))
     assert math.isclose(oracle.gemm_gate(ref * 1.01, ref), 0.01)
+    # with K, the floor is 100 x (K/16) fp32 ulps of rms: 100 * 2048 * 2^-23 = 0.0244 at
+    # K = 32768, and never below 1e-3
+    assert math.isclose(oracle.gemm_gate(ref + [0, 0, 1e-3, 0], ref, 32768),
+                        1e-3 / (100 * 2048 * 2.0 ** -23 * rms))
+    assert oracle.gemm_gate(ref + [0, 0, 1e-3, 0], ref, 16) == oracle.gemm_gate(
+        ref + [0, 0, 1e-3, 0], ref)
+    assert math.isclose(oracle.gemm_gate(ref * 1.01, ref, 32768), 0.01)  # large outputs: relative
 
 
 def test_outlier_quality_ordering():

@@ -466,15 +466,17 @@ gemv_mma(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __restrict_
 // Each group's 8 MMAs run as two independent accumulator chains.
 // Shared-memory layout of gemv_mma_bulk (host and device agree through this).
 struct MmaBulkLayout {
-  uint32_t xf_bytes, sx_bytes, stage_bytes, wbytes, szbytes, ring_off, bar_off, red_off, total;
+  uint32_t xf_bytes, sx_bytes, xq_bytes, stage_bytes, wbytes, szbytes, ring_off, bar_off, red_off,
+      total;
   __host__ __device__ MmaBulkLayout(int M, int K, int wstride, int stages, int NW, int RT) {
     const uint32_t G = K / 128;
     xf_bytes = G * 4 * M * 64;
     sx_bytes = G * 8 * 4;
+    xq_bytes = G * 4 * M * 4;  // per-quarter sums of x, [G][M][4]
     wbytes = 16u * RT * wstride;
     szbytes = 16u * RT * G * 2;
     stage_bytes = wbytes + 2 * szbytes;
-    ring_off = xf_bytes + sx_bytes;
+    ring_off = (xf_bytes + sx_bytes + xq_bytes + 127) / 128 * 128;
     bar_off = ring_off + stages * stage_bytes;
     red_off = bar_off + (2 * stages + 2) * 8;
     total = red_off + 2u * NW * RT * 16 * (M < 2 ? 2 : M) * 4;
@@ -565,40 +567,59 @@ gemv_mma_bulk(const uint16_t* __restrict__ X, int64_t ldx, const uint8_t* __rest
     return;
   }
 
-  // X -> fragment order and per-group token sums; overlaps with the producer's first copies
-  for (int e = threadIdx.x; e < G * 4 * M; e += 32 * NW) {
-    const int g = e / (4 * M);
-    const int Lf = e - g * 4 * M;
-    const int n = Lf >> 2, c = Lf & 3;
-    const uint16_t* xs = X + n * ldx + g * 128 + 32 * c;
-    uint32_t xw[16];
+  // X -> fragment order and per-group token sums; overlaps with the producer's first copies.
+  // A thread issues the loads of up to four of its entries (32 values of one token each) at
+  // once, so the L2 latency is paid once per four entries, and sums each entry's values from
+  // the same registers; the four quarter sums of a group are added in a fixed order below.
+  {
+    float* xq = reinterpret_cast<float*>(smem + L.xf_bytes + L.sx_bytes);  // [G][M][4]
+    const int total = G * 4 * M;
+    for (int e0 = threadIdx.x; e0 < total; e0 += 4 * 32 * NW) {
+      uint4 u[4][4];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint4 u = ld_nc_u4(xs + 8 * v);
-      xw[4 * v] = u.x; xw[4 * v + 1] = u.y; xw[4 * v + 2] = u.z; xw[4 * v + 3] = u.w;
+      for (int j = 0; j < 4; ++j) {
+        const int e = e0 + j * 32 * NW;
+        if (e < total) {
+          const int g = e / (4 * M);
+          const int Lf = e - g * 4 * M;
+          const uint16_t* xs = X + (Lf >> 2) * ldx + g * 128 + 32 * (Lf & 3);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) u[j][v] = ld_nc_u4(xs + 8 * v);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = e0 + j * 32 * NW;
+        if (e < total) {
+          const int g = e / (4 * M);
+          const int Lf = e - g * 4 * M;
+          uint32_t xw[16];
+          float t = 0.0f;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            xw[4 * v] = u[j][v].x; xw[4 * v + 1] = u[j][v].y;
+            xw[4 * v + 2] = u[j][v].z; xw[4 * v + 3] = u[j][v].w;
+            t += ((bf16_lo(u[j][v].x) + bf16_hi(u[j][v].x)) + (bf16_lo(u[j][v].y) + bf16_hi(u[j][v].y))) +
+                 ((bf16_lo(u[j][v].z) + bf16_hi(u[j][v].z)) + (bf16_lo(u[j][v].w) + bf16_hi(u[j][v].w)));
+          }
+          uint32_t frag[16];
+          build_x_fragment(xw, frag);
+          // chunks of quarter c rotated by 2 (c >> 1): a warp's four quarter loads hit four
+          // bank groups
+          uint32_t* dst = xf + (static_cast<size_t>(g) * 4 * M + Lf) * 16;
+          const int xrot = 2 * ((Lf >> 1) & 1);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) dst[(((q >> 2) + xrot) & 3) * 4 + (q & 3)] = frag[q];
+          xq[e] = t;
+        }
+      }
     }
-    uint32_t frag[16];
-    build_x_fragment(xw, frag);
-    // chunks of quarter c rotated by 2 (c >> 1): a warp's four quarter loads hit four bank groups
-    uint32_t* dst = xf + (static_cast<size_t>(g) * 4 * M + Lf) * 16;
-    const int xrot = 2 * ((Lf >> 1) & 1);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) dst[(((j >> 2) + xrot) & 3) * 4 + (j & 3)] = frag[j];
-  }
-  for (int e = threadIdx.x; e < G * 8; e += 32 * NW) {
-    const int g = e >> 3, n = e & 7;
-    float t = 0.0f;
-    if (n < M) {
-      const uint16_t* xs = X + n * ldx + g * 128;
-      uint4 u[16];
-#pragma unroll
-      for (int v = 0; v < 16; ++v) u[v] = ld_nc_u4(xs + 8 * v);
-#pragma unroll
-      for (int v = 0; v < 16; ++v)
-        t += ((bf16_lo(u[v].x) + bf16_hi(u[v].x)) + (bf16_lo(u[v].y) + bf16_hi(u[v].y))) +
-             ((bf16_lo(u[v].z) + bf16_hi(u[v].z)) + (bf16_lo(u[v].w) + bf16_hi(u[v].w)));
+    named_barrier(1, 32 * NW);
+    for (int e = threadIdx.x; e < G * 8; e += 32 * NW) {
+      const int g = e >> 3, n = e & 7;
+      const float* q = xq + (g * M + n) * 4;
+      sxs[e] = n < M ? (q[0] + q[1]) + (q[2] + q[3]) : 0.0f;
     }
-    sxs[e] = t;
   }
   named_barrier(1, 32 * NW);
 

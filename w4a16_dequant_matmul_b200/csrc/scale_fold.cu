@@ -160,8 +160,9 @@ awq_scales_kernel(const float* __restrict__ a_mag, int K, float alpha, float* __
   }
 }
 
-// Four folded weights w * s (float32 products) starting at column k; flags a factor that
-// is not finite and positive.
+// Four folded weights w * s (float32 products) starting at column k. A factor that is not
+// finite and positive is flagged and its column folds to 0, so that it is reported as a bad
+// factor (WQ_ERR_RANGE) rather than through the non-finite products it would make.
 template <typename T>
 __device__ __forceinline__ void fold4(const T* w, const float* s, float v[4], bool& bad_s) {
   float x[4];
@@ -170,8 +171,9 @@ __device__ __forceinline__ void fold4(const T* w, const float* s, float v[4], bo
   const float fs[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    bad_s |= !(fs[i] > 0.0f) || isinf(fs[i]);
-    v[i] = __fmul_rn(x[i], fs[i]);
+    const bool bad = !(fs[i] > 0.0f) || isinf(fs[i]);
+    bad_s |= bad;
+    v[i] = bad ? 0.0f : __fmul_rn(x[i], fs[i]);
   }
 }
 
