@@ -29,6 +29,12 @@ Sources (page title, section):
         exponent a chosen on calibration data by the output error. Also "DL S067 -
         Quantization", section 5 "AWQ intuition" (y = (W diag(s)) (diag(1/s) x), 1/s
         pushed into the previous layer), and "Model Quantization", section 2.2.
+  [GQ]  same page, "GPTQ vs AWQ": GPTQ quantizes one input column at a time and moves each
+        column's rounding error onto the columns not yet quantized through the inverse of
+        the dampened layer-input Hessian H = X^T X + damp * mean(diag) * I, dropping the
+        finished column from the inverse after each step (the Optimal Brain Surgeon
+        update); the quantization grid is fixed before the sweep. Also "DL S067 -
+        Quantization", section 4, and "Model Quantization", section 2.1.
 
 Readings where the pages are silent (each is pinned by a test in tests/test_oracle.py):
   * range includes zero: alpha = min(0, min w), beta = max(0, max w);
@@ -51,6 +57,9 @@ Readings where the pages are silent (each is pinned by a test in tests/test_orac
   * a channel whose statistic is zero (max|X_j| or max|W_j| for SmoothQuant, mean|X_j|
     for AWQ) gets s_j = 1 and is left out of AWQ's normalisation (the pages' formulas
     give 0/0 or 0 there);
+  * GPTQ [GQ]: the grid of each group (S', Z, or the per-row symmetric scale of the
+    page's toy) is computed from the original weights before the sweep, as the toy fixes
+    its per-row scale up front; columns are taken in their natural order;
   * the per-channel mean |X_j| is the column's exact sum (math.fsum, exact whenever the
     sum fits binary64's 53 bits) divided by the row count and rounded once to float32.
 
@@ -78,6 +87,7 @@ __all__ = [
     "outlier_quality", "f32_round", "channel_absmax", "channel_absmean", "smooth_scales",
     "smoothquant_scales", "awq_scales", "fold_input_scales", "fold_weight_f32",
     "quantize_rtn_scaled", "scale_activations_bf16", "awq_search",
+    "gptq_hessian", "gptq_sweep", "gptq_quantize_asym",
 ]
 
 Q4_MIN, Q4_MAX = 0, 15       # asymmetric INT4 integer range [CM]
@@ -525,3 +535,52 @@ def awq_search(W, X, alphas, qdq):
         if best is None or err < best[0]:
             best = (err, a, Q, s)
     return best[2], best[1], best[3]
+
+
+# -------------------------------------------------------------------------- GPTQ [GQ]
+
+def gptq_hessian(X, damp=0.01) -> np.ndarray:
+    """H = X^T X of the calibration activations X [tokens, K], plus damp times the mean of
+    its diagonal on the diagonal (numerical stability) [GQ]."""
+    X = np.asarray(X, dtype=np.float64)
+    H = X.T @ X
+    return H + damp * float(np.mean(np.diag(H))) * np.eye(H.shape[0])
+
+
+def gptq_sweep(W, H, qdq_column):
+    """GPTQ's column sweep [GQ]. W [N, K]; H [K, K] dampened; qdq_column(i, w) returns the
+    quantize-dequantized values of column i for the current values w [N] of that column on
+    a grid fixed before the sweep. Every row sees the same sequence of inverse Hessians, so
+    the rows are swept together: for column i, Q_i = qdq(w_i), the error e = (w_i - Q_i) /
+    Hinv_ii moves onto the later columns as w_j -= e Hinv_ij (j > i), and column i leaves
+    the inverse: Hinv -= Hinv_{:,i} Hinv_{i,:} / Hinv_ii. Returns Q [N, K] (float64)."""
+    Wc = np.array(W, dtype=np.float64, copy=True)
+    Hinv = np.linalg.inv(np.asarray(H, dtype=np.float64))
+    N, K = Wc.shape
+    Q = np.zeros_like(Wc)
+    for i in range(K):
+        Q[:, i] = qdq_column(i, Wc[:, i])
+        err = (Wc[:, i] - Q[:, i]) / Hinv[i, i]
+        Wc[:, i + 1:] -= np.outer(err, Hinv[i, i + 1:])
+        Hinv -= np.outer(Hinv[:, i], Hinv[i, :]) / Hinv[i, i]
+    return Q
+
+
+def gptq_quantize_asym(W, X, group=128, damp=0.01):
+    """GPTQ into the library's INT4 format [GQ][CM]: S' and Z of every group from the
+    original weights (``quantize_rtn_asym``), then the sweep with codes
+    clip(RNE(w/S') + Z, 0, 15) of the updated weights. Returns (codes uint8 [N, K], S, Z)
+    for the unchanged W4A16 kernels."""
+    W = np.asarray(W, dtype=np.float64)
+    _, S, Z = quantize_rtn_asym(W, group)
+    g = group or W.shape[1]
+    codes = np.zeros(W.shape, dtype=np.uint8)
+
+    def qdq(i, w):
+        s, z = S[:, i // g], Z[:, i // g]
+        q = np.clip(np.rint(w / s) + z, Q4_MIN, Q4_MAX)
+        codes[:, i] = q.astype(np.uint8)
+        return s * (q - z)
+
+    gptq_sweep(W, gptq_hessian(X, damp), qdq)
+    return codes, S, Z
