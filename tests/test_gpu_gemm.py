@@ -214,11 +214,11 @@ def test_w8a16_small_m(M):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 4096), (1, 64, 11008), (3, 160, 4096), (8, 128, 2048),
-                                   (64, 136, 1024)])
+                                   (64, 136, 1024), (96, 136, 1024)])
 def test_symmetric_int4_matmul(M, N, K):
     """Symmetric INT4 weights (codes q + 8, Z = 8) through the same matmul kernels: the
-    decode kernels against the exact product, the tensor-core GEMM (M = 64) against the
-    bf16-rounded weights."""
+    decode and skinny kernels (M <= 64) against the exact product, the tensor-core GEMM
+    (M = 96) against the bf16-rounded weights."""
     Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + K)
     Xb = wq_inputs.act_bf16(M, K, seed=M + 9)
     packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb), 4, 128, False)
@@ -227,7 +227,7 @@ def test_symmetric_int4_matmul(M, N, K):
     np.testing.assert_array_equal(gu.to_np(packed), oracle.pack_int4(codes))
     Y = wq.wq_w4a16_gemm(gu.bf16_from_bits(Xb), packed, S, Z, 128)
     assert wq.wq_get_status() == 0
-    mode = "exact" if M <= 32 else "bf16"
+    mode = "exact" if M <= 64 else "bf16"
     Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, mode)
     assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE
 
@@ -262,9 +262,8 @@ def _sampled_rows(N, k, seed):
 def test_70b_skinny_sampled(N, K, M):
     """70B-class decode layers at M = 8 and 32 in the benchmark's configuration (the whole W
     quantized and multiplied on the GPU); the oracle quantizes and multiplies 64 sampled rows,
-    the first and last among them. M = 8 runs as token blocks on the decode kernels, which
-    multiply by the exact S'(q - Z) (one block of 8 at K = 8192, blocks of 2 at K = 28672),
-    as does M = 32 at K = 8192 (four blocks of 8)."""
+    the first and last among them. Both run on the skinny tensor-core kernel, whose
+    integer products with exact activation digits multiply by the exact S'(q - Z)."""
     Wb = wq_inputs.weight_bf16(N, K, 0.015)
     Xb = wq_inputs.act_bf16(M, K)
     packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb))
@@ -273,12 +272,7 @@ def test_70b_skinny_sampled(N, K, M):
     rows = _sampled_rows(N, 64, N + M)
     codes, So, Zo = oracle.quantize_rtn_asym(wq_inputs.bf16_bits_to_f64(Wb[rows]), 128)
     np.testing.assert_array_equal(gu.to_np(packed)[rows], oracle.pack_int4(codes))
-    # M = 32 at K = 28672 runs on the tensor-core GEMM (blocks of 4 tokens do not fit the
-    # decode kernels' shared memory there), which rounds S'(q - Z) to bf16 first; its fp32
-    # accumulation over K sets the gate's floor
-    tc = M == 32 and K == 28672
-    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128,
-                               "bf16" if tc else "exact")
+    Yref = oracle.w4a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), codes, So, Zo, 128, "exact")
     y = gu.bf16_to_f64(Y)[:, rows]
     assert oracle.gemm_gate(y, Yref, K) <= GATE
     assert oracle.rel_frobenius(Yref, y) < 4e-3

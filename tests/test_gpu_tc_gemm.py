@@ -31,12 +31,13 @@ def _run(M, N, K, group=128, seed=0):
     return gu.bf16_to_f64(Y), Yref
 
 
-# shapes that reach the tensor-core kernel (M > 32, or a shape without a fast decode kernel:
-# g != 128 or N % 16 != 0)
-@pytest.mark.parametrize("M,N,K", [(16, 128, 64), (9, 136, 128), (64, 256, 256), (300, 200, 512),
-                                   (257, 384, 1024), (40, 4096, 4096)])
-def test_tc_gemm_parity(M, N, K):
-    y, yref = _run(M, N, K, group=min(K, 128))
+# shapes that reach the tensor-core kernel: M > 64, or M > 8 with g != 128 (the skinny
+# kernel and the fast decode kernels take g = 128 only)
+@pytest.mark.parametrize("M,N,K,group", [(16, 128, 64, 64), (9, 136, 128, 64), (65, 256, 256, 128),
+                                         (300, 200, 512, 128), (257, 384, 1024, 128),
+                                         (40, 4096, 4096, 256), (72, 4096, 4096, 128)])
+def test_tc_gemm_parity(M, N, K, group):
+    y, yref = _run(M, N, K, group=group)
     assert oracle.gemm_gate(y, yref) <= GATE
     assert oracle.rel_frobenius(yref, y) < 4e-3
 
@@ -88,7 +89,7 @@ def test_tc_gemm_deterministic():
     assert torch.equal(Y1, Y2)
 
 
-@pytest.mark.parametrize("M,N,K", [(512, 4096, 11008), (64, 1024, 28672)])
+@pytest.mark.parametrize("M,N,K", [(512, 4096, 11008), (96, 1024, 28672)])
 def test_tc_gemm_long_k_sampled(M, N, K):
     """Long contractions (the 7B down projection in prefill, a 70B-class K): the tensor core's
     fp32 accumulation error grows with K, so the gate's floor is the one derived from K."""

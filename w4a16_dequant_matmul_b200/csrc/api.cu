@@ -212,6 +212,8 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
 // Token counts up to which the decode kernels (in passes of at most 8 tokens, at most
 // kMaxPasses of them) beat the tensor-core GEMM, whose tiles are too few for small M.
 constexpr int64_t kSkinnyMaxM = 32;
+// From this many tokens on (to 64, g = 128) the skinny tensor-core kernel takes the call.
+constexpr int64_t kTcSkinnyMinM = 9;
 constexpr int64_t kMaxPasses = 8;
 
 wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t* packed,
@@ -234,6 +236,15 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
   const int sz_row = group ? (int)(K / group) : 0;
   wq::GemvArgs a{X, ldx, packed, S, Z, (int)(M < 8 ? M : 8), (int)N, (int)K, g, sz_row, Y,
                  ldy, d->status};
+  // kTcSkinnyMinM..64 tokens, g = 128: one pass over the weights on the tensor core
+  if (M >= kTcSkinnyMinM && M <= wq::kSkinnyMaxTokens) {
+    wq::GemvArgs t = a;
+    t.M = static_cast<int>(M);
+    if (wq::tc_skinny_ok(t)) {
+      const cudaError_t e = wq::launch_tc_skinny(t, d->sms, st);
+      if (e != cudaErrorInvalidValue) return from_cuda(e);
+    }
+  }
   // M = 1 beyond the register-loaded kernels' K only where the streaming kernel takes it
   if (M <= kSkinnyMaxM &&
       (M > 1 || K <= wq::gemv_max_k() || wq::gemv_imma_bulk_ok(a) || wq::gemv_tma_ok(a) ||
