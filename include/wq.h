@@ -144,8 +144,16 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
  *   X [M, K] bf16 (ldx), packed/S/Z as produced above with group g (0 = per-tensor),
  *   Y [M, N] bf16 (ldy), fp32 accumulation.
  * Kernel choice by M:
- *   - M <= 32: decode kernels, for M > 8 in passes over blocks of at most 8 tokens (when
- *     some block size needs at most 8 passes; else the tensor-core GEMM). The packed rows
+ *   - 9 <= M <= 64 with g = 128 (K % 128 == 0): the skinny tensor-core kernel, one pass
+ *     over the weights for all tokens. Each token's activations of a group are written as
+ *     exact integers x 2^s below 2^22 (s from the group's largest exponent: exact within 2^14
+ *     of the group's largest |x|, else off by at most 2^-23 of it) in three signed bytes;
+ *     tcgen05 kind::i8 multiplies them with the centred codes q - Z exactly (s32), and
+ *     S' 2^-s is applied per group in fp32, so the product is with the exact S'(q - Z). K
+ *     is split over a thread-block cluster whose partial rows are summed in a fixed order
+ *     (deterministic).
+ *   - otherwise M <= 32: decode kernels, for M > 8 in passes over blocks of at most 8 tokens
+ *     (when some block size needs at most 8 passes; else the tensor-core GEMM). The packed rows
  *     stream through shared memory (bulk copies or TMA boxes) or registers, codes are
  *     decoded in registers (into warp-level bf16 MMAs for g = 128 and N % 16 == 0, else
  *     packed fp32 FMAs), and S' and Z are applied per group in fp32: the product is with
