@@ -235,6 +235,29 @@ wq_status wq_quantize_rtn_scaled(const void* W, wq_dtype w_dtype, int64_t N, int
 wq_status wq_scale_activations(const uint16_t* X, int64_t M, int64_t K, int64_t ldx,
                                const float* s, uint16_t* Xs, int64_t ldxs, void* stream);
 
+/* GPTQ ("LLM Weight Quantization ...", "GPTQ vs AWQ: two ways to choose what error to keep";
+ * "DL S067 - Quantization", section 4): quantize W [N, K] one input column at a time, moving
+ * each column's rounding error onto the columns not yet quantized through the inverse of the
+ * dampened Hessian H = X^T X + damp * mean(diag H) * I of the calibration activations
+ * X [T, K] (bf16, row stride ldx), and dropping the finished column from the inverse
+ * (Optimal Brain Surgeon update). The grid is fixed before the sweep: S' and Z of every
+ * group are those of wq_quantize_rtn_g128 on the original W ({4, g, 1} or {4, g, 0};
+ * params NULL = {4, 128, 1}); only the codes differ. The output format is the same, for the
+ * unchanged matmul kernels. The Hessian, its inverse (Gauss-Jordan, no pivoting) and the
+ * sweep run in float64; one CTA sweeps one row. Requirements: K % 64 == 0, K <= 8192,
+ * T >= 1, 0 <= damp (the page's toy uses 0.01); W as for wq_quantize_rtn_g128; X 2-byte
+ * aligned; workspace of at least wq_gptq_workspace_bytes(N, K) bytes (8 K^2 + 32 K),
+ * 16-byte aligned, no initial contents. A Hessian that is not positive definite (for
+ * example damp = 0 with fewer calibration rows than K) or a non-finite weight sets
+ * WQ_ERR_NONFINITE in the status word. Offline: 2K launches of O(K^2) each plus the sweep
+ * (measured 17 ms for 1024 x 1024 with 256 calibration rows, 0.56 s for 4096 x 4096 with
+ * 512). */
+size_t wq_gptq_workspace_bytes(int64_t N, int64_t K);
+wq_status wq_quantize_gptq(const void* W, wq_dtype w_dtype, int64_t N, int64_t K, int64_t ldw,
+                           const uint16_t* X, int64_t T, int64_t ldx, double damp,
+                           const wq_qparams* params, uint8_t* packed, uint16_t* S, uint16_t* Z,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronize `stream`, then return and clear the current device's status word:
  * WQ_OK, or the first of WQ_ERR_NONFINITE / WQ_ERR_RANGE / WQ_ERR_TIMEOUT recorded by a
  * kernel since the last call; WQ_ERR_CUDA if the synchronization itself failed. */

@@ -566,13 +566,16 @@ def gptq_sweep(W, H, qdq_column):
     return Q
 
 
-def gptq_quantize_asym(W, X, group=128, damp=0.01):
+def gptq_quantize_asym(W, X, group=128, damp=0.01, sym=False):
     """GPTQ into the library's INT4 format [GQ][CM]: S' and Z of every group from the
-    original weights (``quantize_rtn_asym``), then the sweep with codes
-    clip(RNE(w/S') + Z, 0, 15) of the updated weights. Returns (codes uint8 [N, K], S, Z)
-    for the unchanged W4A16 kernels."""
+    original weights (``quantize_rtn_asym``, or with ``sym`` the symmetric grid in its stored
+    form, Z = 8), then the sweep with codes clip(RNE(w/S') + Z, 0, 15) of the updated
+    weights. Returns (codes uint8 [N, K], S, Z) for the unchanged W4A16 kernels."""
     W = np.asarray(W, dtype=np.float64)
-    _, S, Z = quantize_rtn_asym(W, group)
+    if sym:
+        _, S, Z = sym_int4_storage(*quantize_rtn_sym_int4(W, group))
+    else:
+        _, S, Z = quantize_rtn_asym(W, group)
     g = group or W.shape[1]
     codes = np.zeros(W.shape, dtype=np.uint8)
 

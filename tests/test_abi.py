@@ -149,6 +149,25 @@ def test_scale_folding_argument_checks(lib):
     assert a(FAKE, 2, 64, 64, FAKE, FAKE, 72, None) == UNSUP             # in place, other ld
 
 
+def test_gptq_argument_checks(lib):
+    g = lib.wq_quantize_gptq
+    ws = lib.wq_gptq_workspace_bytes(64, 256)
+    assert ws == 8 * 256 * 256 + 32 * 256
+    args = lambda **kw: (kw.get("W", FAKE), kw.get("dt", wq.WQ_BF16), kw.get("N", 64),
+                         kw.get("K", 256), kw.get("ldw", 256), kw.get("X", FAKE), kw.get("T", 32),
+                         kw.get("ldx", 256), kw.get("damp", 0.01), kw.get("qp", None), FAKE, FAKE,
+                         FAKE, kw.get("ws", FAKE), kw.get("wsb", ws), None)
+    assert g(*args(N=0)) == OK
+    assert g(*args(X=None)) == NULL
+    assert g(*args(T=0)) == SHAPE
+    assert g(*args(K=96, ldw=96, ldx=96)) == SHAPE         # K % 64
+    assert g(*args(damp=-1.0)) == SHAPE
+    assert g(*args(wsb=ws - 8)) == SHAPE                  # workspace too small
+    assert g(*args(qp=_qp(8, 256, 0))) == UNSUP
+    assert g(*args(K=16384, ldw=16384, ldx=16384, wsb=1 << 40)) == UNSUP  # K > 8192
+    assert g(*args(ws=ODD)) == ALIGN
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="host without a GPU only")
 def test_valid_call_without_device_reports_nodevice(lib):
     """A call that passes every host check but finds no sm_100 device fails loudly

@@ -44,6 +44,10 @@ def test_gptq_with_diagonal_hessian_is_rtn():
     c_rtn, S, Z = oracle.quantize_rtn_asym(W, 128)
     c_gptq, S2, Z2 = oracle.gptq_quantize_asym(W, X, 128)
     assert np.array_equal(c_rtn, c_gptq) and np.array_equal(S, S2) and np.array_equal(Z, Z2)
+    q, Ss = oracle.quantize_rtn_sym_int4(W, 128)
+    c_sym, S3, Z3 = oracle.gptq_quantize_asym(W, X, 128, sym=True)
+    assert np.array_equal(c_sym.astype(np.int16) - 8, q) and np.array_equal(S3, Ss)
+    assert np.all(Z3 == 8.0)
     Q = oracle.gptq_sweep(W, oracle.gptq_hessian(X), _toy_grid(W))
     scale = np.abs(W).max(axis=1, keepdims=True) / 3
     np.testing.assert_array_equal(Q, np.clip(np.rint(W / scale), -4, 3) * scale)

@@ -17,6 +17,7 @@ Functions carry the C names:
     wq_awq_scales(a_mag, alpha) -> s
     wq_quantize_rtn_scaled(W, s, group=128, zero_point=True) -> (packed, S, Z)
     wq_scale_activations(X, s) -> X / s
+    wq_quantize_gptq(W, X, group=128, zero_point=True, damp=0.01) -> (packed, S, Z)
     wq_get_status() -> int
 S and Z are returned as torch.float16 tensors (binary16 bit patterns in the C ABI).
 """
@@ -35,7 +36,7 @@ __all__ = [
     "wq_pack_int4", "wq_dequant", "wq_w4a16_gemm",
     "wq_w8a16_gemm", "wq_get_status", "wq_selftest_bounded_wait",
     "wq_channel_stat", "wq_smooth_scales", "wq_awq_scales", "wq_quantize_rtn_scaled",
-    "wq_scale_activations",
+    "wq_scale_activations", "wq_quantize_gptq", "wq_gptq_workspace_bytes",
     "WQ_F32", "WQ_BF16", "WQ_F16", "WQ_U8", "WQ_I8", "WQ_STAT_ABSMAX", "WQ_STAT_ABSMEAN",
 ]
 
@@ -84,6 +85,9 @@ _SIGNATURES = {
     "wq_quantize_rtn_scaled": (_I32, [_P, _I32, _I64, _I64, _I64, _P, ctypes.POINTER(_QParams),
                                       _P, _P, _P, _P]),
     "wq_scale_activations": (_I32, [_P, _I64, _I64, _I64, _P, _P, _I64, _P]),
+    "wq_gptq_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "wq_quantize_gptq": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I64, _I64, ctypes.c_double,
+                                ctypes.POINTER(_QParams), _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "wq_selftest_bounded_wait": (_I32, [ctypes.c_uint64, _I32, _P]),
 }
 
@@ -417,6 +421,37 @@ def wq_scale_activations(X, s, out=None, stream=None):
                                         _stream(stream))
     _check(st, "wq_scale_activations")
     return out
+
+
+def wq_gptq_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().wq_gptq_workspace_bytes(N, K))
+
+
+def wq_quantize_gptq(W, X, group: int = 128, zero_point: bool = True, damp: float = 0.01,
+                     workspace=None, stream=None):
+    """GPTQ of W [N, K] (float32 or bfloat16) on calibration activations X [T, K] (bfloat16):
+    returns (packed uint8 [N, K/2], S fp16 [N, K/g], Z fp16 [N, K/g]) in the RTN format."""
+    import torch
+
+    N, K = W.shape
+    T = X.shape[0]
+    ldw = _rows(W, "W")
+    ldx = _rows(X, "X")
+    dev = W.device
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    S = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    Z = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    nbytes = wq_gptq_workspace_bytes(N, K)
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=dev)
+    p = _QParams(4, group, 1 if zero_point else 0)
+    with _on_device(W):
+        st = lib().wq_quantize_gptq(_ptr(W), _w_dtype(W), N, K, ldw, _ptr(X), T, ldx,
+                                    float(damp), ctypes.byref(p), _ptr(packed), _ptr(S), _ptr(Z),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream))
+    _check(st, "wq_quantize_gptq")
+    return packed, S, Z
 
 
 def wq_selftest_bounded_wait(limit_ns: int = 20_000_000, spin: bool = True, stream=None) -> None:

@@ -383,6 +383,44 @@ wq_status wq_scale_activations(const uint16_t* X, int64_t M, int64_t K, int64_t 
                                                 static_cast<cudaStream_t>(stream)));
 }
 
+size_t wq_gptq_workspace_bytes(int64_t N, int64_t K) {
+  (void)N;
+  return K > 0 ? wq::gptq_workspace_bytes(K) : 0;
+}
+
+wq_status wq_quantize_gptq(const void* W, wq_dtype w_dtype, int64_t N, int64_t K, int64_t ldw,
+                           const uint16_t* X, int64_t T, int64_t ldx, double damp,
+                           const wq_qparams* params, uint8_t* packed, uint16_t* S, uint16_t* Z,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  const wq_qparams p = params ? *params : wq_qparams{4, 128, 1};
+  if (N < 0 || K < 0 || T < 0) return WQ_ERR_SHAPE;
+  if (w_dtype != WQ_F32 && w_dtype != WQ_BF16) return WQ_ERR_DTYPE;
+  if (p.w_bit != 4 || (p.zero_point != 0 && p.zero_point != 1)) return WQ_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return WQ_OK;
+  if (!W || !X || !packed || !S || !Z || !workspace) return WQ_ERR_NULL;
+  if (!fits_int(N) || !fits_int(K) || !fits_int(T) || T == 0 || K % 64 != 0 || ldw < K ||
+      ldx < K || !(damp >= 0.0 && damp <= 1e6))
+    return WQ_ERR_SHAPE;
+  if (p.group < 32 || p.group % 32 != 0 || K % p.group != 0) return WQ_ERR_SHAPE;
+  if (K > wq::gptq_max_k()) return WQ_ERR_UNSUPPORTED;
+  const size_t es = w_dtype == WQ_F32 ? 4 : 2;
+  if (!aligned(W, 16) || (ldw * es) % 16 != 0 || !aligned(packed, 16) || !aligned(S, 2) ||
+      !aligned(Z, 2) || !aligned(X, 2) || !aligned(workspace, 16))
+    return WQ_ERR_ALIGN;
+  if (workspace_bytes < wq::gptq_workspace_bytes(K)) return WQ_ERR_SHAPE;
+  const DeviceInfo* d = device_info();
+  if (!d) return WQ_ERR_NODEVICE;
+  if (!on_current_device({W, X, packed, S, Z, workspace})) return WQ_ERR_DEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = w_dtype == WQ_BF16;
+  // the grid: round-to-nearest S' and Z of the original weights (its codes are replaced)
+  cudaError_t e = wq::launch_quant_asym(W, bf16, ldw, (int)N, (int)K, p.group, packed, S, Z,
+                                        p.zero_point == 0, d->status, d->sms, st);
+  if (e != cudaSuccess) return WQ_ERR_CUDA;
+  return from_cuda(wq::launch_gptq(W, bf16, ldw, (int)N, (int)K, p.group, X, ldx, (int)T, damp,
+                                   packed, S, Z, workspace, d->status, d->sms, st));
+}
+
 wq_status wq_selftest_bounded_wait(uint64_t limit_ns, int32_t spin, void* stream) {
   if (limit_ns < 1000u || limit_ns > 1000000000u) return WQ_ERR_SHAPE;
   const DeviceInfo* d = device_info();

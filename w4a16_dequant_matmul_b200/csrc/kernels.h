@@ -92,6 +92,14 @@ cudaError_t launch_scale_activations(const uint16_t* X, int64_t ldx, int M, int 
                                      const float* s, uint16_t* Xs, int64_t ldxs, int sms,
                                      cudaStream_t st);
 
+// GPTQ sweep on a fixed grid (gptq.cu): workspace of gptq_workspace_bytes(K) bytes.
+size_t gptq_workspace_bytes(int64_t K);
+int gptq_max_k();
+cudaError_t launch_gptq(const void* W, bool bf16, int64_t ldw, int N, int K, int group,
+                        const uint16_t* X, int64_t ldx, int T, double damp, uint8_t* packed,
+                        const uint16_t* S, const uint16_t* Z, void* workspace, unsigned* status,
+                        int sms, cudaStream_t st);
+
 // One CTA whose single bounded mbarrier wait runs out (selftest.cu).
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, bool spin, unsigned* status,
                                          cudaStream_t st);
