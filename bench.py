@@ -558,6 +558,41 @@ def run_gpu(args):
         prefill = f"unavailable: {e}"
     secondary["prefill"] = prefill
 
+    # ---- secondary: offline quantization variants on one 7B-class layer (11008 x 4096):
+    # scale folding (SmoothQuant factors from 64 calibration tokens, the folded quantizer, X/s)
+    # and GPTQ (512 calibration tokens; 1024 x 1024 and the full layer's 4096 x 4096 slice)
+    offline = {}
+    try:
+        Wt = (torch.randn(11008, 4096, device=dev) * 0.02).to(torch.bfloat16)
+        Xc = torch.randn(64, 4096, device=dev).to(torch.bfloat16)
+        sf = wq.wq_smooth_scales(wq.wq_channel_stat(Xc, wq.WQ_STAT_ABSMAX),
+                                 wq.wq_channel_stat(Wt, wq.WQ_STAT_ABSMAX), 0.5)
+        pk, s, z = wq.wq_quantize_rtn_scaled(Wt, sf)
+        us = graph_time_us(lambda: wq.wq_quantize_rtn_scaled(Wt, sf, packed=pk, S=s, Z=z), 5)
+        fold_b = Wt.numel() * 2 + 4 * 4096 + pk.numel() + 4 * s.numel()
+        offline["quantize_rtn_scaled_11008x4096"] = {"us": round(us, 1),
+                                                     "GB/s": round(fold_b / us / 1e3, 1)}
+        g_times = {}
+        for (n, k) in ((1024, 1024), (4096, 4096)):
+            Wg = Wt[:n, :k].contiguous()
+            Xg = torch.randn(512, k, device=dev).to(torch.bfloat16)
+            ws = torch.empty(wq.wq_gptq_workspace_bytes(n, k), dtype=torch.uint8, device=dev)
+            wq.wq_quantize_gptq(Wg, Xg, workspace=ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            wq.wq_quantize_gptq(Wg, Xg, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            g_times[f"{n}x{k}_T512_ms"] = round(e0.elapsed_time(e1), 2)
+            del Wg, Xg, ws
+        offline["gptq"] = g_times
+        assert wq.wq_get_status() == 0
+        del Wt, Xc, sf, pk, s, z
+    except Exception as e:
+        offline = f"unavailable: {e}"
+    secondary["offline_quantizers"] = offline
+
     # ---- e2e: through the public API with host buffers per step: the step's three X rows
     # arrive in one pinned buffer (one H2D copy) and its three Y rows leave in one (one D2H)
     kx = [x.shape[1] for x in X]

@@ -144,7 +144,9 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
  *   X [M, K] bf16 (ldx), packed/S/Z as produced above with group g (0 = per-tensor),
  *   Y [M, N] bf16 (ldy), fp32 accumulation.
  * Kernel choice by M:
- *   - 9 <= M <= 64 with g = 128 (K % 128 == 0): the skinny tensor-core kernel, one pass
+ *   - 9 <= M <= 64 with g = 128 (K % 128 == 0), and 3 <= M <= 8 where the decode kernels
+ *     below would pass over the weights more than once (rows too long for blocks of M
+ *     tokens): the skinny tensor-core kernel, one pass
  *     over the weights for all tokens. Each token's activations of a group are written as
  *     exact integers x 2^s below 2^22 (s from the group's largest exponent: exact within 2^14
  *     of the group's largest |x|, else off by at most 2^-23 of it) in three signed bytes;

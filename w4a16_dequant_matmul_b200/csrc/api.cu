@@ -212,7 +212,8 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
 // Token counts up to which the decode kernels (in passes of at most 8 tokens, at most
 // kMaxPasses of them) beat the tensor-core GEMM, whose tiles are too few for small M.
 constexpr int64_t kSkinnyMaxM = 32;
-// From this many tokens on (to 64, g = 128) the skinny tensor-core kernel takes the call.
+// From this many tokens on (to 64, g = 128) the skinny tensor-core kernel takes the call;
+// below it only where the decode kernels would pass over the weights more than once.
 constexpr int64_t kTcSkinnyMinM = 9;
 constexpr int64_t kMaxPasses = 8;
 
@@ -236,11 +237,13 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
   const int sz_row = group ? (int)(K / group) : 0;
   wq::GemvArgs a{X, ldx, packed, S, Z, (int)(M < 8 ? M : 8), (int)N, (int)K, g, sz_row, Y,
                  ldy, d->status};
-  // kTcSkinnyMinM..64 tokens, g = 128: one pass over the weights on the tensor core
-  if (M >= kTcSkinnyMinM && M <= wq::kSkinnyMaxTokens) {
+  // 3..64 tokens, g = 128: one pass over the weights on the tensor core, from
+  // kTcSkinnyMinM tokens on, or wherever the decode kernels would need more than one pass
+  // over blocks of tokens (long rows at small M)
+  if (M >= 3 && M <= wq::kSkinnyMaxTokens) {
     wq::GemvArgs t = a;
     t.M = static_cast<int>(M);
-    if (wq::tc_skinny_ok(t)) {
+    if (wq::tc_skinny_ok(t) && (M >= kTcSkinnyMinM || wq::gemv_fast_block(a) < M)) {
       const cudaError_t e = wq::launch_tc_skinny(t, d->sms, st);
       if (e != cudaErrorInvalidValue) return from_cuda(e);
     }
