@@ -178,9 +178,11 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
                         int32_t group, uint16_t* Y, int64_t ldy, void* stream);
 
 /* W8A16 matmul with INT8 symmetric per-channel weights: codes int8 [N, K], S [N]
- * binary16; Y = X (s' q)^T, fp32 accumulation, bf16 out. M <= 8 runs on CUDA cores with
- * the exact s' q; larger M on the tensor-core GEMM (s' q rounded to bf16). Same
- * requirements as wq_w4a16_gemm. */
+ * binary16; Y = X (s' q)^T, fp32 accumulation, bf16 out. 3 <= M <= 64 with K % 128 == 0
+ * runs on the skinny tensor-core kernel (tcgen05 kind::i8 on the s8 codes as stored and the
+ * exact activation digits described for wq_w4a16_gemm; s' applied to the finished row), one
+ * pass over the weights; M <= 2 (and other M <= 8) on CUDA cores with the exact s' q; larger
+ * M on the tensor-core GEMM (s' q rounded to bf16). Same requirements as wq_w4a16_gemm. */
 wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t* codes,
                         const uint16_t* S, int64_t N, int64_t K, uint16_t* Y, int64_t ldy,
                         void* stream);

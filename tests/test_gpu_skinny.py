@@ -1,6 +1,7 @@
-"""Parity of the skinny tensor-core W4A16 kernel (9 to 64 tokens, g = 128: tcgen05 kind::i8
-on the centred codes q - Z and exact activation digits, split-K over a cluster) with the
-float64 oracle on the exact dequantized weights S'(q - Z), through the C ABI.
+"""Parity of the skinny tensor-core kernel (tcgen05 kind::i8 on exact activation digits,
+split-K over a cluster) with the float64 oracle, through the C ABI: W4A16 (9 to 64 tokens,
+g = 128, centred codes q - Z) on the exact dequantized weights S'(q - Z), and W8A16 (1 to 64
+tokens, the s8 codes copied as they are) on the exact s' q.
 
 Cases span one group (K = 128, no split), ragged row counts (a partial 128-row tile), every
 token-count class (16, 32, 64 columns per digit plane) with ragged M, long K (70B-class), and
@@ -106,3 +107,34 @@ def test_skinny_nonfinite_activation_propagates():
     Xk = wq_inputs.bf16_bits_to_f64(Xb[keep])
     Yref = oracle.w4a16_matmul(Xk, codes, So, Zo, 128, "exact")
     assert oracle.gemm_gate(Y[keep], Yref, K) <= GATE
+
+
+@pytest.mark.parametrize("M", [1, 3, 8, 16, 17, 40, 64])
+@pytest.mark.parametrize("N,K", [(300, 512), (1024, 2048)])
+def test_skinny_w8a16_parity(M, N, K):
+    Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=50 + N)
+    Xb = wq_inputs.act_bf16(M, K, seed=51 + M)
+    q, S, _ = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb), 8, K, False)
+    Y = wq.wq_w8a16_gemm(gu.bf16_from_bits(Xb), q, S)
+    assert wq.wq_get_status() == 0
+    qo, so = oracle.quantize_sym_int8_per_channel(wq_inputs.bf16_bits_to_f64(Wb))
+    np.testing.assert_array_equal(gu.to_np(q), qo)
+    Yref = oracle.w8a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), qo, so, "exact")
+    y = gu.bf16_to_f64(Y)
+    assert oracle.gemm_gate(y, Yref, K) <= GATE
+    assert oracle.rel_frobenius(Yref, y) < 4e-3
+
+
+def test_skinny_w8a16_7b_shapes_sampled():
+    """W8A16 decode at M = 1 on the 7B-class shapes (sampled rows)."""
+    for (N, K) in wq_inputs.SHAPES_7B:
+        Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + 1)
+        Xb = wq_inputs.act_bf16(1, K, seed=K + 1)
+        q, S, _ = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb), 8, K, False)
+        Y = wq.wq_w8a16_gemm(gu.bf16_from_bits(Xb), q, S)
+        assert wq.wq_get_status() == 0
+        rows = np.sort(np.random.default_rng(N).choice(N, 48, replace=False))
+        rows[0], rows[-1] = 0, N - 1
+        qo, so = oracle.quantize_sym_int8_per_channel(wq_inputs.bf16_bits_to_f64(Wb[rows]))
+        Yref = oracle.w8a16_matmul(wq_inputs.bf16_bits_to_f64(Xb), qo, so, "exact")
+        assert oracle.gemm_gate(gu.bf16_to_f64(Y)[:, rows], Yref, K) <= GATE

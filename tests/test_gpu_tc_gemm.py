@@ -67,7 +67,7 @@ def test_tc_gemm_prefill_shape_sampled():
     assert oracle.gemm_gate(y, Yref) <= GATE
 
 
-@pytest.mark.parametrize("M,N,K", [(24, 128, 256), (2048, 1024, 4096)])
+@pytest.mark.parametrize("M,N,K", [(96, 128, 256), (2048, 1024, 4096)])
 def test_tc_w8a16(M, N, K):
     Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=3)
     Xb = wq_inputs.act_bf16(M, K, seed=4)

@@ -65,6 +65,9 @@ cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st);
 constexpr int kSkinnyMaxTokens = 64;
 bool tc_skinny_ok(const GemvArgs& a);
 cudaError_t launch_tc_skinny(const GemvArgs& a, int sms, cudaStream_t st);
+// The same for W8A16: a.P = int8 codes [N, K], a.S = per-row scales [N], a.Z unused.
+bool tc_skinny8_ok(const GemvArgs& a);
+cudaError_t launch_tc_skinny8(const GemvArgs& a, int sms, cudaStream_t st);
 
 // Small-M W8A16 (symmetric INT8 per output channel) on CUDA cores.
 struct Gemv8Args {

@@ -55,7 +55,11 @@ constexpr int kPrepWarps = 8, kEpiWarps = 4;
 constexpr uint64_t kLimitNs = 2000000000ull;
 constexpr uint32_t kTmemCols = 512;
 
-template <int MT>
+// kW8: INT8 symmetric per-channel weights (W8A16). The s8 codes are the A operand as they
+// are: the producer copies each [128 rows x 128 k] box with TMA straight into the operand
+// stage in the 128-byte-swizzled layout, so there is no expansion role; the row's scale
+// s' is applied once, to the finished row.
+template <int MT, bool kW8>
 struct SkCfg {
   static constexpr int NC = 3 * MT;                      // accumulator columns per group
   static constexpr int kBBytes = NC * kGK;               // digit planes, 128-byte rows
@@ -66,14 +70,15 @@ struct SkCfg {
   static constexpr int kOpBytes = (kMetaOff + kMetaBytes + 1023) / 1024 * 1024;
   static constexpr int kOpStages = MT <= 16 ? 6 : (MT <= 32 ? 4 : 3);
   // load ring (packed codes | activations), freed once expansion and digits have read it
-  static constexpr int kXOff = kRawBytes;
-  static constexpr int kLdBytes = (kRawBytes + kXBytes + 1023) / 1024 * 1024;
+  static constexpr int kRawLd = kW8 ? 0 : kRawBytes;
+  static constexpr int kXOff = kRawLd;
+  static constexpr int kLdBytes = (kRawLd + kXBytes + 1023) / 1024 * 1024;
   static constexpr int kLdStages = MT <= 16 ? 6 : (MT <= 32 ? 5 : 3);
   static constexpr int kBufs = MT <= 32 ? 4 : 2;          // TMEM accumulators in flight
   static constexpr int kChunk = MT <= 16 ? 16 : 8;         // tokens per epilogue TMEM load
   // code-expansion warps: 8 (one half row per thread), or 4 (two) where the epilogue's MT
   // accumulators need the registers of a smaller block
-  static constexpr int kDecWarps = MT <= 32 ? 8 : 4;
+  static constexpr int kDecWarps = kW8 ? 0 : (MT <= 32 ? 8 : 4);
   static constexpr int kThreads = 32 * (2 + kDecWarps + kPrepWarps + kEpiWarps);
   static_assert(kBufs * NC <= static_cast<int>(kTmemCols), "TMEM");
   static_assert(kRows * MT * 4 <= kOpBytes, "cluster partials fit in operand stage 0");
@@ -83,7 +88,7 @@ struct SkCfg {
 struct SkBars {
   uint64_t ld_full[6];   // TMA: a load stage's codes and activations landed
   uint64_t ld_empty[6];  // expansion and digit warps have read the load stage
-  uint64_t a_full[6];    // code expansion into the operand stage done
+  uint64_t a_full[6];    // code expansion (W8A16: the TMA copy) into the operand stage done
   uint64_t b_full[6];    // digit planes and 2^-s done
   uint64_t op_empty[6];  // operand stage free: the MMAs are done and the epilogue read 2^-s
   uint64_t acc_full[4];  // a group's accumulator is complete
@@ -93,9 +98,9 @@ struct SkBars {
   volatile int abort;
 };
 
-template <int MT>
+template <int MT, bool kW8>
 constexpr size_t sk_smem_bytes() {
-  using C = SkCfg<MT>;
+  using C = SkCfg<MT, kW8>;
   return 1024 + C::kOpStages * C::kOpBytes + C::kLdStages * C::kLdBytes + sizeof(SkBars);
 }
 
@@ -120,12 +125,12 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
 }
 
-template <int MT>
-__global__ void __launch_bounds__(SkCfg<MT>::kThreads, 1)
+template <int MT, bool kW8>
+__global__ void __launch_bounds__(SkCfg<MT, kW8>::kThreads, 1)
 tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int M, int N,
                  int K, uint16_t* __restrict__ Y, int64_t ldy, unsigned* status) {
-  using C = SkCfg<MT>;
+  using C = SkCfg<MT, kW8>;
   constexpr int NC = C::NC, kOpStages = C::kOpStages, kLdStages = C::kLdStages,
                 kBufs = C::kBufs;
   constexpr int kDecWarps = C::kDecWarps, kThreads = C::kThreads;
@@ -155,7 +160,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       mbar_init(&sb->ld_empty[s], kDecWarps + kPrepWarps);
     }
     for (int s = 0; s < kOpStages; ++s) {
-      mbar_init(&sb->a_full[s], kDecWarps);
+      mbar_init(&sb->a_full[s], kW8 ? 1 : kDecWarps);
       mbar_init(&sb->b_full[s], kPrepWarps);
       mbar_init(&sb->op_empty[s], 1 + kEpiWarps);
     }
@@ -185,18 +190,32 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int it = 0;
-      for (; it < ng && !sb->abort; ++it) {
+      int nld = 0, na = 0;  // load-ring fills and (W8A16) operand-stage code copies issued
+      for (int it = 0; it < ng && !sb->abort; ++it) {
         const int s = it % kLdStages;
         const uint32_t u = it / kLdStages;
         if (u > 0 && !sk_wait(&sb->ld_empty[s], (u - 1) & 1u, sb, status)) break;
-        mbar_arrive_expect_tx(&sb->ld_full[s], kRawBytes + C::kXBytes);
-        tma_load_2d(ldst(s), &tmW, (g0 + it) * (kGK / 2), n0, &sb->ld_full[s]);
+        mbar_arrive_expect_tx(&sb->ld_full[s], C::kRawLd + C::kXBytes);
+        if constexpr (!kW8) tma_load_2d(ldst(s), &tmW, (g0 + it) * (kGK / 2), n0, &sb->ld_full[s]);
         tma_load_2d(ldst(s) + C::kXOff, &tmX, (g0 + it) * kGK, 0, &sb->ld_full[s]);
+        ++nld;
+        if constexpr (kW8) {  // the s8 codes straight into the operand stage (swizzled)
+          const int os = it % kOpStages;
+          const uint32_t ou = it / kOpStages;
+          if (ou > 0 && !sk_wait(&sb->op_empty[os], (ou - 1) & 1u, sb, status)) break;
+          mbar_arrive_expect_tx(&sb->a_full[os], kABytes);
+          tma_load_2d(opst(os), &tmW, (g0 + it) * kGK, n0, &sb->a_full[os]);
+          ++na;
+        }
       }
-      for (int s = 0; s < kLdStages && s < it; ++s) {  // no copy left in flight on exit
-        const uint32_t last = (it - 1 - s) / kLdStages;
+      // no copy left in flight on exit: wait (bounded) for the last fill of every stage
+      for (int s = 0; s < kLdStages && s < nld; ++s) {
+        const uint32_t last = (nld - 1 - s) / kLdStages;
         if (!mbar_wait_bounded(&sb->ld_full[s], last & 1u, kLimitNs)) set_status(status, kStTimeout);
+      }
+      for (int s = 0; s < kOpStages && s < na; ++s) {
+        const uint32_t last = (na - 1 - s) / kOpStages;
+        if (!mbar_wait_bounded(&sb->a_full[s], last & 1u, kLimitNs)) set_status(status, kStTimeout);
       }
     }
   } else if (warp == 1) {
@@ -225,6 +244,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       if (!mbar_wait_bounded(&sb->done, 0, kLimitNs)) set_status(status, kStTimeout);
     }
   } else if (warp < 2 + kDecWarps) {
+    if constexpr (!kW8) {
     // --------------------------------------------------------------- code expansion
     // thread t takes the half rows (row, half) = pair >> 1, pair & 1 for pairs t, t + 32
     // kDecWarps, ...: a quarter-warp reads 256 contiguous bytes of the raw tile, and each
@@ -288,6 +308,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       }
 #pragma unroll
       for (int pp = 0; pp < kPairs; ++pp) zc[pp] = zn[pp];
+    }
     }
   } else if (warp < 2 + kDecWarps + kPrepWarps) {
     // ------------------------------------------------------------- activation digits
@@ -368,8 +389,10 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
     const bool live = n < N;
     const int64_t szrow = static_cast<int64_t>(live ? n : 0) * G;
     // S' of this row two groups ahead (the loads stay in flight across iterations)
+    // (W8A16: the row's scale is applied once, to the finished row)
     auto ld_s = [&](int it) {
-      return it < ng && live ? f16_bits_to_f32(ld_nc_u16(S + szrow + g0 + it)) : 0.0f;
+      if constexpr (kW8) return live ? 1.0f : 0.0f;
+      else return it < ng && live ? f16_bits_to_f32(ld_nc_u16(S + szrow + g0 + it)) : 0.0f;
     };
     float s0 = ld_s(0), s1 = ld_s(1);
     for (int it = 0; it < ng && !sb->abort; ++it) {
@@ -441,6 +464,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       for (int r = 1; r < 8; ++r)
         if (r < csize) t += v[r];  // rank order
       if (n0 + row < N) {
+        if constexpr (kW8) t *= f16_bits_to_f32(ld_nc_u16(S + n0 + row));
         __nv_bfloat16 hv = __float2bfloat16_rn(t);
         Y[static_cast<int64_t>(m) * ldy + n0 + row] = *reinterpret_cast<uint16_t*>(&hv);
       }
@@ -473,7 +497,7 @@ int pick_split(int tiles, int G, int sms) {
   return best;
 }
 
-template <int MT>
+template <int MT, bool kW8>
 cudaError_t launch_mt(const GemvArgs& a, const CUtensorMap& map, int sms, cudaStream_t st) {
   // activations as [M rows][K] bf16: boxes of 128 k x MT tokens (rows past M read as zero);
   // kept per thread for the last few activation buffers (decode loops reuse them)
@@ -503,8 +527,8 @@ cudaError_t launch_mt(const GemvArgs& a, const CUtensorMap& map, int sms, cudaSt
     xnext = (xnext + 1) % kXCache;
     xmap = &e.map;
   }
-  auto kern = tc_skinny_kernel<MT>;
-  const size_t smem = sk_smem_bytes<MT>();
+  auto kern = tc_skinny_kernel<MT, kW8>;
+  const size_t smem = sk_smem_bytes<MT, kW8>();
   static std::atomic<bool> attr[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -518,7 +542,7 @@ cudaError_t launch_mt(const GemvArgs& a, const CUtensorMap& map, int sms, cudaSt
   const int cs = pick_split(tiles, G, sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * cs);
-  cfg.blockDim = dim3(SkCfg<MT>::kThreads);
+  cfg.blockDim = dim3(SkCfg<MT, kW8>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attrs[2];
@@ -536,43 +560,68 @@ cudaError_t launch_mt(const GemvArgs& a, const CUtensorMap& map, int sms, cudaSt
 
 }  // namespace
 
-bool tc_skinny_ok(const GemvArgs& a) {
-  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  return a.M >= 1 && a.M <= kSkinnyMaxTokens && a.group == 128 && a.sz_row == a.K / 128 &&
-         a.K % 128 == 0 && a.N >= 1 && a.ldx % 8 == 0 && al16(a.X) && al16(a.P);
-}
+namespace {
 
-cudaError_t launch_tc_skinny(const GemvArgs& a, int sms, cudaStream_t st) {
-  if (!tc_skinny_ok(a)) return cudaErrorInvalidValue;
-  // packed codes as [N rows][K/2 bytes]: boxes of 64 bytes (one group) x 128 rows; the map
-  // is kept per thread for the last few weight matrices (decode calls repeat)
+// Tensor map of the weights, kept per thread for the last few matrices (decode calls
+// repeat): INT4 packed codes as [N rows][K/2 bytes] in boxes of 64 bytes (one group) x 128
+// rows; INT8 codes as [N rows][K bytes] in 128-byte-swizzled boxes of 128 x 128 bytes.
+const CUtensorMap* weight_map(const void* P, int N, int K, bool w8) {
   struct MapEntry {
     const void* p;
     int n, k;
+    bool w8;
     CUtensorMap map;
   };
   constexpr int kMapCache = 16;
   thread_local MapEntry cache[kMapCache];
   thread_local int next_slot = 0;
-  const CUtensorMap* map = nullptr;
   for (const MapEntry& e : cache)
-    if (e.p == a.P && e.n == a.N && e.k == a.K) map = &e.map;
-  if (!map) {
-    MapEntry& e = cache[next_slot];
-    e.p = nullptr;
-    if (!make_map_2d(&e.map, a.P, static_cast<uint64_t>(a.K / 2), static_cast<uint64_t>(a.N),
-                     static_cast<uint64_t>(a.K / 2), kGK / 2, kRows, false,
-                     CU_TENSOR_MAP_DATA_TYPE_UINT8))
-      return cudaErrorInvalidValue;
-    e.p = a.P;
-    e.n = a.N;
-    e.k = a.K;
-    next_slot = (next_slot + 1) % kMapCache;
-    map = &e.map;
-  }
-  if (a.M <= 16) return launch_mt<16>(a, *map, sms, st);
-  if (a.M <= 32) return launch_mt<32>(a, *map, sms, st);
-  return launch_mt<64>(a, *map, sms, st);
+    if (e.p == P && e.n == N && e.k == K && e.w8 == w8) return &e.map;
+  MapEntry& e = cache[next_slot];
+  e.p = nullptr;
+  const uint64_t row = w8 ? static_cast<uint64_t>(K) : static_cast<uint64_t>(K / 2);
+  if (!make_map_2d(&e.map, P, row, static_cast<uint64_t>(N), row, w8 ? kGK : kGK / 2, kRows,
+                   w8, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+    return nullptr;
+  e.p = P;
+  e.n = N;
+  e.k = K;
+  e.w8 = w8;
+  next_slot = (next_slot + 1) % kMapCache;
+  return &e.map;
+}
+
+template <bool kW8>
+cudaError_t launch_skinny(const GemvArgs& a, int sms, cudaStream_t st) {
+  const CUtensorMap* map = weight_map(a.P, a.N, a.K, kW8);
+  if (!map) return cudaErrorInvalidValue;
+  if (a.M <= 16) return launch_mt<16, kW8>(a, *map, sms, st);
+  if (a.M <= 32) return launch_mt<32, kW8>(a, *map, sms, st);
+  return launch_mt<64, kW8>(a, *map, sms, st);
+}
+
+bool skinny_common_ok(const GemvArgs& a) {
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  return a.M >= 1 && a.M <= kSkinnyMaxTokens && a.K % 128 == 0 && a.N >= 1 &&
+         a.ldx % 8 == 0 && al16(a.X) && al16(a.P);
+}
+
+}  // namespace
+
+bool tc_skinny_ok(const GemvArgs& a) {
+  return skinny_common_ok(a) && a.group == 128 && a.sz_row == a.K / 128;
+}
+
+cudaError_t launch_tc_skinny(const GemvArgs& a, int sms, cudaStream_t st) {
+  if (!tc_skinny_ok(a)) return cudaErrorInvalidValue;
+  return launch_skinny<false>(a, sms, st);
+}
+
+bool tc_skinny8_ok(const GemvArgs& a) { return skinny_common_ok(a); }
+
+cudaError_t launch_tc_skinny8(const GemvArgs& a, int sms, cudaStream_t st) {
+  if (!tc_skinny8_ok(a)) return cudaErrorInvalidValue;
+  return launch_skinny<true>(a, sms, st);
 }
 
 }  // namespace wq
