@@ -1,7 +1,8 @@
 """Parity of the skinny tensor-core kernel (tcgen05 kind::i8 on exact activation digits,
 split-K over a cluster) with the float64 oracle, through the C ABI: W4A16 (9 to 64 tokens,
-g = 128, centred codes q - Z) on the exact dequantized weights S'(q - Z), and W8A16 (1 to 64
-tokens, the s8 codes copied as they are) on the exact s' q.
+g = 128, centred codes q - Z) on the exact dequantized weights S'(q - Z), and W8A16 (3 to 64
+tokens, the s8 codes copied as they are) on the exact s' q. The W8A16 cases also cover one
+token, which runs on the row kernel, against the same exact product.
 
 Cases span one group (K = 128, no split), ragged row counts (a partial 128-row tile), every
 token-count class (16, 32, 64 columns per digit plane) with ragged M, long K (70B-class), and
@@ -125,11 +126,13 @@ def test_skinny_w8a16_parity(M, N, K):
     assert oracle.rel_frobenius(Yref, y) < 4e-3
 
 
-def test_skinny_w8a16_7b_shapes_sampled():
-    """W8A16 decode at M = 1 on the 7B-class shapes (sampled rows)."""
+@pytest.mark.parametrize("M", [1, 4])
+def test_skinny_w8a16_7b_shapes_sampled(M):
+    """W8A16 decode on the 7B-class shapes (sampled rows): M = 1 on the row kernel, M = 4
+    on the skinny kernel."""
     for (N, K) in wq_inputs.SHAPES_7B:
         Wb = wq_inputs.weight_bf16(N, K, 0.02, seed=N + 1)
-        Xb = wq_inputs.act_bf16(1, K, seed=K + 1)
+        Xb = wq_inputs.act_bf16(M, K, seed=K + 1)
         q, S, _ = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb), 8, K, False)
         Y = wq.wq_w8a16_gemm(gu.bf16_from_bits(Xb), q, S)
         assert wq.wq_get_status() == 0
