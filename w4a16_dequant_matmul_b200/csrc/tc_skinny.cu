@@ -333,14 +333,9 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         const int m = item >> 3, c = item & 7;  // token, 16-k chunk (8 lanes per token)
         const uint4 u0 = lds128(xs_s + m * 256 + 32 * c), u1 = lds128(xs_s + m * 256 + 32 * c + 16);
         const uint32_t wds[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-        uint32_t xb[16];
         uint32_t e2 = 0;  // exponent fields of both halves, maximised pairwise
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          xb[2 * i] = wds[i] & 0xFFFFu;
-          xb[2 * i + 1] = wds[i] >> 16;
-          e2 = __vmaxu2(e2, wds[i] & 0x7F807F80u);
-        }
+        for (int i = 0; i < 8; ++i) e2 = __vmaxu2(e2, wds[i] & 0x7F807F80u);
         uint32_t e = max(e2 & 0xFFFFu, e2 >> 16) >> 7;
         e = max(e, __shfl_xor_sync(0xffffffffu, e, 1));
         e = max(e, __shfl_xor_sync(0xffffffffu, e, 2));
@@ -352,13 +347,28 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
 #pragma unroll
           for (int i = 0; i < 16; ++i) z[i] = 0u;
         } else {
-          // s = 21 - (exponent of the largest |x|), so |x 2^s| < 2^22
+          // s = 21 - (exponent of the largest |x|), so |x 2^s| < 2^22. Two values per packed
+          // FMA: x 2^s + 1.5 2^23 with one rounding (x 2^s is exact; for groups below 2^-106,
+          // 2^s is applied as 2^100 2^(s - 100)), i.e. x_int in the low bits; then the
+          // balanced signed bytes as in the integer decode path.
           const int sc = 21 - (static_cast<int>(e < 1u ? 1u : e) - 127);
           const bool split = sc > 127;
-          const uint32_t p2b = split ? 0u : static_cast<uint32_t>(sc + 127) << 7;
-          const float f1 = split ? pow2i(100) : 0.0f, f2 = split ? pow2i(sc - 100) : 0.0f;
+          const float f1 = pow2i(100);
+          const float sf = split ? pow2i(sc - 100) : pow2i(sc);
+          const float2 sf2 = make_float2(sf, sf), mg2 = make_float2(kImmaMagic, kImmaMagic);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) z[i] = digits_of(xb[i], p2b, split, f1, f2);
+          for (int i = 0; i < 8; ++i) {
+            float2 v = make_float2(__uint_as_float(wds[i] << 16),
+                                   __uint_as_float(wds[i] & 0xFFFF0000u));
+            if (split) {
+              v.x *= f1;
+              v.y *= f1;
+            }
+            const float2 t = __ffma2_rn(v, sf2, mg2);
+            constexpr uint32_t kOff = 0x808080u - static_cast<uint32_t>(kImmaMagicBits);
+            z[2 * i] = (static_cast<uint32_t>(__float_as_int(t.x)) + kOff) ^ 0x808080u;
+            z[2 * i + 1] = (static_cast<uint32_t>(__float_as_int(t.y)) + kOff) ^ 0x808080u;
+          }
           p = pow2i(-sc);
         }
         // digit plane i: bytes i of z[0..15], 16 consecutive k of token m
