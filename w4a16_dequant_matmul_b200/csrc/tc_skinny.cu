@@ -27,7 +27,8 @@
 //                tile;
 //   next 8 warps activation digits: 8 threads per token, 16 k each: the group's exponent,
 //                the digit planes into the swizzled B tile, and 2^-s;
-//   last 4 warps epilogue: thread = TMEM lane = weight row; reads the three digit planes of
+//   last 4 (8 at MT = 64) warps  epilogue: thread = TMEM lane = weight row (at MT = 64 two
+//                warps per lane quarter, each for half the tokens); reads the three digit planes of
 //                the group's accumulator, combines them, applies S' 2^-s, accumulates fp32.
 // Every mbarrier wait is bounded (2 s): on a timeout the kernel records kStTimeout, every role
 // leaves its loop, the producer waits (bounded) for its copies, the MMA lane for its last
@@ -51,7 +52,7 @@ constexpr int kRows = 128;                 // weight rows per tile (MMA M)
 constexpr int kGK = 128;                   // k per group (one stage)
 constexpr int kRawBytes = kRows * kGK / 2;  // packed codes of a stage: 8 KB
 constexpr int kABytes = kRows * kGK;        // u8 codes, 128-byte rows: 16 KB
-constexpr int kPrepWarps = 8, kEpiWarps = 4;
+constexpr int kPrepWarps = 8;
 constexpr uint64_t kLimitNs = 2000000000ull;
 constexpr uint32_t kTmemCols = 512;
 
@@ -79,6 +80,10 @@ struct SkCfg {
   // code-expansion warps: 8 (one half row per thread), or 4 (two) where the epilogue's MT
   // accumulators need the registers of a smaller block
   static constexpr int kDecWarps = kW8 ? 0 : (MT <= 32 ? 8 : 4);
+  // epilogue warps: one per TMEM lane quarter, or two at MT = 64, each then keeping the
+  // accumulators of half the tokens (32 registers instead of 64)
+  static constexpr int kEpiWarps = MT <= 32 ? 4 : 8;
+  static constexpr int kEpiTok = MT / (kEpiWarps / 4);  // tokens per epilogue thread
   static constexpr int kThreads = 32 * (2 + kDecWarps + kPrepWarps + kEpiWarps);
   static_assert(kBufs * NC <= static_cast<int>(kTmemCols), "TMEM");
   static_assert(kRows * MT * 4 <= kOpBytes, "cluster partials fit in operand stage 0");
@@ -133,7 +138,8 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   using C = SkCfg<MT, kW8>;
   constexpr int NC = C::NC, kOpStages = C::kOpStages, kLdStages = C::kLdStages,
                 kBufs = C::kBufs;
-  constexpr int kDecWarps = C::kDecWarps, kThreads = C::kThreads;
+  constexpr int kDecWarps = C::kDecWarps, kThreads = C::kThreads, kEpiWarps = C::kEpiWarps;
+  constexpr int kEpiTok = C::kEpiTok;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -183,9 +189,9 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   if (threadIdx.x == 0) pdl_launch_dependents();
   pdl_wait();  // X, the codes, S and Z are read only after the previous kernel completed
 
-  float acc[MT];
+  float acc[kEpiTok];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+  for (int m = 0; m < kEpiTok; ++m) acc[m] = 0.0f;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -395,6 +401,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
     // ---------------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes 32 quarter .. + 31 (this warp's window)
     const int row = quarter * 32 + lane;
+    const int tb = ((warp - (2 + kDecWarps + kPrepWarps)) >> 2) * kEpiTok;  // first token
     const int n = n0 + row;
     const bool live = n < N;
     const int64_t szrow = static_cast<int64_t>(live ? n : 0) * G;
@@ -415,26 +422,27 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * NC;
       constexpr int CH = C::kChunk;
 #pragma unroll
-      for (int mc = 0; mc < MT / CH; ++mc) {
+      for (int mc = 0; mc < kEpiTok / CH; ++mc) {
         uint32_t d0[CH], d1[CH], d2[CH];
+        const uint32_t col = tb + CH * mc;
         if constexpr (CH == 16) {
-          tmem_ld16(taddr + 0 * MT + CH * mc, d0);
-          tmem_ld16(taddr + 1 * MT + CH * mc, d1);
-          tmem_ld16(taddr + 2 * MT + CH * mc, d2);
+          tmem_ld16(taddr + 0 * MT + col, d0);
+          tmem_ld16(taddr + 1 * MT + col, d1);
+          tmem_ld16(taddr + 2 * MT + col, d2);
         } else {
-          tmem_ld8(taddr + 0 * MT + CH * mc, d0);
-          tmem_ld8(taddr + 1 * MT + CH * mc, d1);
-          tmem_ld8(taddr + 2 * MT + CH * mc, d2);
+          tmem_ld8(taddr + 0 * MT + col, d0);
+          tmem_ld8(taddr + 1 * MT + col, d1);
+          tmem_ld8(taddr + 2 * MT + col, d2);
         }
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
-          const int m = CH * mc + i;
-          // |D_i| < 2^18: digits 0 and 1 combine exactly in 32 bits
+          const int j = CH * mc + i;
+          // |D_i| < 2^21 (2^18 with INT4 codes): digits 0 and 1 combine exactly in 32 bits
           const int d01 = static_cast<int>(d0[i]) + 256 * static_cast<int>(d1[i]);
           const float v = fmaf(65536.0f, static_cast<float>(static_cast<int>(d2[i])),
                                static_cast<float>(d01));
-          acc[m] = fmaf(sv * meta[m], v, acc[m]);
+          acc[j] = fmaf(sv * meta[tb + j], v, acc[j]);
         }
       }
       tc_fence_before();
@@ -456,8 +464,9 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   float* part = reinterpret_cast<float*>(base);  // [MT][kRows]
   if (warp >= 2 + kDecWarps + kPrepWarps) {
     const int row = (warp & 3) * 32 + lane;
+    const int tb = ((warp - (2 + kDecWarps + kPrepWarps)) >> 2) * kEpiTok;
 #pragma unroll
-    for (int m = 0; m < MT; ++m) part[m * kRows + row] = acc[m];
+    for (int j = 0; j < kEpiTok; ++j) part[(tb + j) * kRows + row] = acc[j];
   }
   cluster.sync();
   if (!sb->abort) {
