@@ -202,3 +202,43 @@ def test_folded_w4a16_matmul_matches_oracle(method, M):
     mode = "bf16" if M > 32 else "exact"
     Yref = oracle.w4a16_matmul(Xs_o, codes, So, Zo, 128, mode=mode)
     assert oracle.gemm_gate(gu.bf16_to_f64(Y), Yref) <= GATE
+
+
+def test_awq_exponent_search_composes_from_gpu_calls():
+    """AWQ's search on the page's calibration toy, in the library's INT4 g128 format, from
+    the GPU calls: mean |X_j| (wq_channel_stat), the factors for each exponent
+    (wq_awq_scales), the folded codes (wq_quantize_rtn_scaled). Each step matches the oracle
+    (factors within a float32 ulp, codes bit for bit on the same factors), and every exponent's
+    calibration output error is the oracle's, so the exponent chosen is the oracle's best."""
+    W, X_cal, _ = wq_inputs.calibration_toy_tensors()
+    W32 = W.astype(np.float32)
+    Xb = wq_inputs.to_bf16_bits(X_cal)
+    X = wq_inputs.bf16_bits_to_f64(Xb)
+    a_gpu = wq.wq_channel_stat(gu.bf16_from_bits(Xb), wq.WQ_STAT_ABSMEAN)
+    np.testing.assert_array_equal(gu.to_np(a_gpu).astype(np.float64), oracle.channel_absmean(X))
+    Y = oracle.matmul_f64(X, W32.astype(np.float64))
+    errs = []
+    for a in np.linspace(0, 1, 11):
+        a32 = float(np.float32(a))
+        s = wq.wq_awq_scales(a_gpu, a32)
+        s64 = gu.to_np(s).astype(np.float64)
+        _f32_close(s64, oracle.awq_scales(oracle.channel_absmean(X), a32)
+                   .astype(np.float32).astype(np.float64))
+        packed, S, Z = wq.wq_quantize_rtn_scaled(gu.f32(W32), s)
+        assert wq.wq_get_status() == 0
+        codes, So, Zo = oracle.quantize_rtn_scaled(W32.astype(np.float64), s64, 128)
+        np.testing.assert_array_equal(gu.to_np(packed), oracle.pack_int4(codes))
+        Q = oracle.dequant_asym(codes, So, Zo, 128) / s64          # fold 1/s back
+        errs.append(oracle.rel_frobenius(Y, oracle.matmul_f64(X, Q)))
+    # the oracle's own search (float64 factors) scores every exponent alike, within 1e-3
+    # relative: the two agree on the best exponent up to near ties
+    qdq = lambda Ws: oracle.dequant_asym(*oracle.quantize_rtn_asym(
+        Ws.astype(np.float32).astype(np.float64), 128), 128)
+    errs_or = []
+    for a in np.linspace(0, 1, 11):
+        Qo, _, _ = oracle.awq_search(W32.astype(np.float64), X, [a], qdq)
+        errs_or.append(oracle.rel_frobenius(Y, oracle.matmul_f64(X, Qo)))
+    np.testing.assert_allclose(errs, errs_or, rtol=1e-3)
+    best = int(np.argmin(errs))
+    assert errs_or[best] <= min(errs_or) * (1 + 1e-3)
+    assert errs[best] < 0.95 * errs[0]  # scaling helps against round-to-nearest (exponent 0)
