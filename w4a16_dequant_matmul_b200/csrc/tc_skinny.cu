@@ -52,34 +52,48 @@ constexpr int kRows = 128;                 // weight rows per tile (MMA M)
 constexpr int kGK = 128;                   // k per group (one stage)
 constexpr int kRawBytes = kRows * kGK / 2;  // packed codes of a stage: 8 KB
 constexpr int kABytes = kRows * kGK;        // u8 codes, 128-byte rows: 16 KB
-constexpr int kPrepWarps = 8;
 constexpr uint64_t kLimitNs = 2000000000ull;
 constexpr uint32_t kTmemCols = 512;
+// The expansion and epilogue roles load Z and S' of a group this many groups ahead, into
+// register rings: a group's work is much shorter than a round trip to DRAM.
+constexpr int kAhead = 8;
 
-// kW8: INT8 symmetric per-channel weights (W8A16). The s8 codes are the A operand as they
-// are: the producer copies each [128 rows x 128 k] box with TMA straight into the operand
-// stage in the 128-byte-swizzled layout, so there is no expansion role; the row's scale
-// s' is applied once, to the finished row.
-template <int MT, bool kW8>
+// Operand modes:
+//   kModeI4Dig  INT4 codes: centred codes q - Z as s8 x activation digit planes (kind::i8).
+//   kModeW8     INT8 symmetric per-channel weights (W8A16): the s8 codes are the A operand
+//               as they are. The producer copies each [128 rows x 128 k] box with TMA
+//               straight into the operand stage in the 128-byte-swizzled layout, so there is
+//               no expansion role; the row's scale s' is applied once, to the finished row.
+//   kModeI4Bf   INT4 codes: centred codes q - Z as bf16 (exact: integers in [-15, 15]) x the
+//               activations as they are, bf16 (kind::f16 with fp32 accumulation; every
+//               product is exact in fp32). The producer copies X with TMA straight into the
+//               operand stage (two 128-byte-swizzled boxes of 64 k per group), so there is no
+//               digit role, and the epilogue applies S' to one accumulator column per token.
+enum SkMode { kModeI4Dig = 0, kModeW8 = 1, kModeI4Bf = 2 };
+
+template <int MT, int kMode>
 struct SkCfg {
-  static constexpr int NC = 3 * MT;                      // accumulator columns per group
-  static constexpr int kBBytes = NC * kGK;               // digit planes, 128-byte rows
-  static constexpr int kXBytes = MT * kGK * 2;           // the group's activations, bf16
-  static constexpr int kMetaBytes = MT * 4;              // per token: 2^-s
-  // operand ring (A | B | 2^-s), freed by the MMA and the epilogue
-  static constexpr int kMetaOff = kABytes + kBBytes;
+  static constexpr bool kW8m = kMode == kModeW8, kBf = kMode == kModeI4Bf;
+  static constexpr int NC = kBf ? MT : 3 * MT;           // accumulator columns per group
+  static constexpr int kA = kBf ? 2 * kABytes : kABytes;  // A operand bytes (bf16: two atoms)
+  static constexpr int kBBytes = kBf ? MT * kGK * 2 : NC * kGK;  // X tile or digit planes
+  static constexpr int kXBytes = kBf ? 0 : MT * kGK * 2;  // activations in the load ring
+  static constexpr int kMetaBytes = kBf ? 0 : MT * 4;     // per token: 2^-s
+  // operand ring (A | B | 2^-s), freed by the MMA (and the epilogue, which reads 2^-s)
+  static constexpr int kMetaOff = kA + kBBytes;
   static constexpr int kOpBytes = (kMetaOff + kMetaBytes + 1023) / 1024 * 1024;
-  static constexpr int kOpStages = MT <= 16 ? 6 : (MT <= 32 ? 4 : 3);
+  static constexpr int kOpStages = kBf ? 4 : (MT <= 16 ? 6 : (MT <= 32 ? 4 : 3));
   // load ring (packed codes | activations), freed once expansion and digits have read it
-  static constexpr int kRawLd = kW8 ? 0 : kRawBytes;
+  static constexpr int kRawLd = kW8m ? 0 : kRawBytes;
   static constexpr int kXOff = kRawLd;
   static constexpr int kLdBytes = (kRawLd + kXBytes + 1023) / 1024 * 1024;
-  static constexpr int kLdStages = MT <= 16 ? 6 : (MT <= 32 ? 5 : 3);
-  static constexpr int kBufs = MT <= 32 ? 4 : 2;          // TMEM accumulators in flight
-  static constexpr int kChunk = MT <= 16 ? 16 : 8;         // tokens per epilogue TMEM load
+  static constexpr int kLdStages = MT <= 16 ? 6 : (MT <= 32 ? (kBf ? 6 : 5) : 3);
+  static constexpr int kBufs = (kBf || MT <= 32) ? 4 : 2;  // TMEM accumulators in flight
+  static constexpr int kChunk = (kBf || MT <= 16) ? 16 : 8;  // tokens per epilogue TMEM load
   // code-expansion warps: 8 (one half row per thread), or 4 (two) where the epilogue's MT
   // accumulators need the registers of a smaller block
-  static constexpr int kDecWarps = kW8 ? 0 : (MT <= 32 ? 8 : 4);
+  static constexpr int kDecWarps = kW8m ? 0 : ((kBf || MT <= 32) ? 8 : 4);
+  static constexpr int kPrepWarps = kBf ? 0 : 8;  // activation digits
   // epilogue warps: one per TMEM lane quarter, or two at MT = 64, each then keeping the
   // accumulators of half the tokens (32 registers instead of 64)
   static constexpr int kEpiWarps = MT <= 32 ? 4 : 8;
@@ -88,6 +102,7 @@ struct SkCfg {
   static_assert(kBufs * NC <= static_cast<int>(kTmemCols), "TMEM");
   static_assert(kRows * MT * 4 <= kOpBytes, "cluster partials fit in operand stage 0");
   static_assert(kOpStages <= 6 && kLdStages <= 6, "barrier arrays");
+  static_assert(kEpiTok % kChunk == 0, "epilogue chunks");
 };
 
 struct SkBars {
@@ -103,15 +118,20 @@ struct SkBars {
   volatile int abort;
 };
 
-template <int MT, bool kW8>
+template <int MT, int kMode>
 constexpr size_t sk_smem_bytes() {
-  using C = SkCfg<MT, kW8>;
+  using C = SkCfg<MT, kMode>;
   return 1024 + C::kOpStages * C::kOpBytes + C::kLdStages * C::kLdBytes + sizeof(SkBars);
 }
 
 // Instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major, M = 128, N = nc.
 __host__ __device__ constexpr uint32_t idesc_i8(int nc) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nc >> 3) << 17) |
+         (static_cast<uint32_t>(kRows >> 4) << 24);
+}
+// Instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both K-major, M = 128, N = nc.
+__host__ __device__ constexpr uint32_t idesc_bf16(int nc) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nc >> 3) << 17) |
          (static_cast<uint32_t>(kRows >> 4) << 24);
 }
 
@@ -125,17 +145,26 @@ __device__ __forceinline__ bool sk_wait(uint64_t* bar, uint32_t parity, SkBars* 
   return false;
 }
 
+// a - b on two packed bf16 values (exact where the difference is representable)
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 d =
+      __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&d);
+}
+
 // 16-byte chunk c (0..7) of row r in a K-major tile with 128-byte rows, 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
 }
 
-template <int MT, bool kW8>
-__global__ void __launch_bounds__(SkCfg<MT, kW8>::kThreads, 1)
+template <int MT, int kMode>
+__global__ void __launch_bounds__(SkCfg<MT, kMode>::kThreads, 1)
 tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const uint16_t* __restrict__ S, const uint16_t* __restrict__ Zp, int M, int N,
                  int K, uint16_t* __restrict__ Y, int64_t ldy, unsigned* status) {
-  using C = SkCfg<MT, kW8>;
+  using C = SkCfg<MT, kMode>;
+  constexpr bool kW8m = C::kW8m, kBf = C::kBf;
+  constexpr int kPrepWarps = C::kPrepWarps, kA = C::kA;
   constexpr int NC = C::NC, kOpStages = C::kOpStages, kLdStages = C::kLdStages,
                 kBufs = C::kBufs;
   constexpr int kDecWarps = C::kDecWarps, kThreads = C::kThreads, kEpiWarps = C::kEpiWarps;
@@ -166,9 +195,9 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       mbar_init(&sb->ld_empty[s], kDecWarps + kPrepWarps);
     }
     for (int s = 0; s < kOpStages; ++s) {
-      mbar_init(&sb->a_full[s], kW8 ? 1 : kDecWarps);
-      mbar_init(&sb->b_full[s], kPrepWarps);
-      mbar_init(&sb->op_empty[s], 1 + kEpiWarps);
+      mbar_init(&sb->a_full[s], kW8m ? 1 : kDecWarps);
+      mbar_init(&sb->b_full[s], kBf ? 1 : kPrepWarps);
+      mbar_init(&sb->op_empty[s], kBf ? 1 : 1 + kEpiWarps);
     }
     for (int b = 0; b < kBufs; ++b) {
       mbar_init(&sb->acc_full[b], 1);
@@ -196,22 +225,29 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int nld = 0, na = 0;  // load-ring fills and (W8A16) operand-stage code copies issued
+      int nld = 0, nop = 0;  // load-ring fills and operand-stage copies issued
       for (int it = 0; it < ng && !sb->abort; ++it) {
         const int s = it % kLdStages;
         const uint32_t u = it / kLdStages;
         if (u > 0 && !sk_wait(&sb->ld_empty[s], (u - 1) & 1u, sb, status)) break;
         mbar_arrive_expect_tx(&sb->ld_full[s], C::kRawLd + C::kXBytes);
-        if constexpr (!kW8) tma_load_2d(ldst(s), &tmW, (g0 + it) * (kGK / 2), n0, &sb->ld_full[s]);
-        tma_load_2d(ldst(s) + C::kXOff, &tmX, (g0 + it) * kGK, 0, &sb->ld_full[s]);
+        if constexpr (!kW8m) tma_load_2d(ldst(s), &tmW, (g0 + it) * (kGK / 2), n0, &sb->ld_full[s]);
+        if constexpr (!kBf) tma_load_2d(ldst(s) + C::kXOff, &tmX, (g0 + it) * kGK, 0, &sb->ld_full[s]);
         ++nld;
-        if constexpr (kW8) {  // the s8 codes straight into the operand stage (swizzled)
+        if constexpr (kW8m || kBf) {
+          // straight into the operand stage (swizzled): the s8 codes (A) or the activations (B)
           const int os = it % kOpStages;
           const uint32_t ou = it / kOpStages;
           if (ou > 0 && !sk_wait(&sb->op_empty[os], (ou - 1) & 1u, sb, status)) break;
-          mbar_arrive_expect_tx(&sb->a_full[os], kABytes);
-          tma_load_2d(opst(os), &tmW, (g0 + it) * kGK, n0, &sb->a_full[os]);
-          ++na;
+          if constexpr (kW8m) {
+            mbar_arrive_expect_tx(&sb->a_full[os], kABytes);
+            tma_load_2d(opst(os), &tmW, (g0 + it) * kGK, n0, &sb->a_full[os]);
+          } else {
+            mbar_arrive_expect_tx(&sb->b_full[os], C::kBBytes);
+            tma_load_2d(opst(os) + kA, &tmX, (g0 + it) * kGK, 0, &sb->b_full[os]);
+            tma_load_2d(opst(os) + kA + MT * 128, &tmX, (g0 + it) * kGK + 64, 0, &sb->b_full[os]);
+          }
+          ++nop;
         }
       }
       // no copy left in flight on exit: wait (bounded) for the last fill of every stage
@@ -219,9 +255,10 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         const uint32_t last = (nld - 1 - s) / kLdStages;
         if (!mbar_wait_bounded(&sb->ld_full[s], last & 1u, kLimitNs)) set_status(status, kStTimeout);
       }
-      for (int s = 0; s < kOpStages && s < na; ++s) {
-        const uint32_t last = (na - 1 - s) / kOpStages;
-        if (!mbar_wait_bounded(&sb->a_full[s], last & 1u, kLimitNs)) set_status(status, kStTimeout);
+      for (int s = 0; s < kOpStages && s < nop; ++s) {
+        const uint32_t last = (nop - 1 - s) / kOpStages;
+        uint64_t* bar = kW8m ? &sb->a_full[s] : &sb->b_full[s];
+        if (!mbar_wait_bounded(bar, last & 1u, kLimitNs)) set_status(status, kStTimeout);
       }
     }
   } else if (warp == 1) {
@@ -237,12 +274,21 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
           break;
         tc_fence_after();
         const uint8_t* a = opst(s);
-        const uint8_t* bt = opst(s) + kABytes;
+        const uint8_t* bt = opst(s) + kA;
         const uint32_t d = tmem + b * NC;
+        if constexpr (kBf) {
+          // K = 16 per MMA; k 0..63 in the first 128-byte-swizzled atom of each operand
 #pragma unroll
-        for (int k = 0; k < kGK / 32; ++k)
-          tc_mma_i8(d, sw128_desc(a + 32 * k), sw128_desc(bt + 32 * k), idesc_i8(NC),
-                    k != 0 ? 1u : 0u);
+          for (int k = 0; k < kGK / 16; ++k)
+            tc_mma(d, sw128_desc(a + (k >> 2) * kABytes + 32 * (k & 3)),
+                   sw128_desc(bt + (k >> 2) * (MT * 128) + 32 * (k & 3)), idesc_bf16(NC),
+                   k != 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int k = 0; k < kGK / 32; ++k)
+            tc_mma_i8(d, sw128_desc(a + 32 * k), sw128_desc(bt + 32 * k), idesc_i8(NC),
+                      k != 0 ? 1u : 0u);
+        }
         tc_commit(&sb->op_empty[s]);
         tc_commit(&sb->acc_full[b]);
       }
@@ -250,35 +296,56 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       if (!mbar_wait_bounded(&sb->done, 0, kLimitNs)) set_status(status, kStTimeout);
     }
   } else if (warp < 2 + kDecWarps) {
-    if constexpr (!kW8) {
+    if constexpr (!kW8m) {
     // --------------------------------------------------------------- code expansion
-    // thread t takes the half rows (row, half) = pair >> 1, pair & 1 for pairs t, t + 32
-    // kDecWarps, ...: a quarter-warp reads 256 contiguous bytes of the raw tile, and each
-    // 16-byte store of the eight lands in a distinct slot
+    // s8 codes: thread t takes the half rows (row, half) = pair >> 1, pair & 1 for pairs
+    // t, t + 32 kDecWarps, ...: a quarter-warp reads 256 contiguous bytes of the raw tile,
+    // and each 16-byte store of the eight lands in a distinct slot. bf16 codes (half h of a
+    // row is the row of atom h): the 8 threads of a quarter-warp take 8 consecutive rows
+    // (distinct store slots) and both halves (reads spread over 4 slots); the quarter-warp
+    // after it takes the same rows' other halves.
     constexpr int kPairs = 256 / (32 * kDecWarps);
     const int t = threadIdx.x - 64;
     const int G = K / kGK;
+    auto pair_rh = [&](int pp, int& r, int& h) {
+      const int pr = t + 32 * kDecWarps * pp;
+      if constexpr (kBf) {
+        r = 8 * (pr >> 4) + (pr & 7);
+        h = ((pr >> 3) & 1) ^ ((pr >> 1) & 1);
+      } else {
+        r = pr >> 1;
+        h = pr & 1;
+      }
+    };
     int64_t zrow[kPairs];
 #pragma unroll
     for (int pp = 0; pp < kPairs; ++pp) {
-      const int n = n0 + ((t + 32 * kDecWarps * pp) >> 1);
+      int r, h;
+      pair_rh(pp, r, h);
+      const int n = n0 + r;
       zrow[pp] = n < N ? static_cast<int64_t>(n) * G : -1;  // rows past N: codes and Z are 0
     }
-    // Z of the rows one group ahead (the loads stay in flight across an iteration)
+    // Z of the rows, in every byte (s8) or as 128 + Z in both bf16 halves
     auto ld_z = [&](int it, uint32_t (&z4)[kPairs]) {
 #pragma unroll
-      for (int pp = 0; pp < kPairs; ++pp)
-        z4[pp] = it < ng && zrow[pp] >= 0
-                     ? static_cast<uint32_t>(f16_bits_to_f32(ld_nc_u16(Zp + zrow[pp] + g0 + it))) *
-                           0x01010101u
-                     : 0u;
+      for (int pp = 0; pp < kPairs; ++pp) {
+        const uint32_t z =
+            it < ng && zrow[pp] >= 0
+                ? static_cast<uint32_t>(f16_bits_to_f32(ld_nc_u16(Zp + zrow[pp] + g0 + it)))
+                : 0u;
+        z4[pp] = kBf ? z * 0x00010001u + 0x43004300u : z * 0x01010101u;
+      }
     };
-    uint32_t zc[kPairs], zn[kPairs];
-    ld_z(0, zc);
-    for (int it = 0; it < ng && !sb->abort; ++it) {
+    uint32_t zq[kAhead][kPairs];
+#pragma unroll
+    for (int j = 0; j < kAhead; ++j) ld_z(j, zq[j]);
+    for (int it0 = 0; it0 < ng && !sb->abort; it0 += kAhead) {
+#pragma unroll
+    for (int j = 0; j < kAhead; ++j) {
+      const int it = it0 + j;
+      if (it >= ng || sb->abort) break;
       const int ls = it % kLdStages, os = it % kOpStages;
       const uint32_t ou = it / kOpStages;
-      ld_z(it + 1, zn);
       if (!sk_wait(&sb->ld_full[ls], (it / kLdStages) & 1u, sb, status) ||
           (ou > 0 && !sk_wait(&sb->op_empty[os], (ou - 1) & 1u, sb, status)))
         break;
@@ -286,25 +353,43 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       const uint32_t at = smem_u32(opst(os));
 #pragma unroll
       for (int pp = 0; pp < kPairs; ++pp) {
-        const int pr = t + 32 * kDecWarps * pp;
-        const int r = pr >> 1, h = pr & 1;
+        int r, h;
+        pair_rh(pp, r, h);
         const uint4 p0 = lds128(raw + r * 64 + 32 * h), p1 = lds128(raw + r * 64 + 32 * h + 16);
         const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        uint32_t o[16];
+        const uint32_t zb = zq[j][pp];  // Z of this group (ring slot j)
+        if constexpr (kBf) {
+          // word c = codes 8c .. 8c + 7 of the half row = 16-byte chunk c of its atom row.
+          // bf16 pair e: byte e of the word (low half) and of the word >> 4 (high half), low
+          // nibbles kept and 0x4300 set: 128 + code exactly; minus 128 + Z: q - Z exactly.
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          // codes + 128 in every byte (no byte can borrow from its neighbour below)
-          const uint32_t lo = (w[q] & 0x0F0F0F0Fu) | 0x80808080u;
-          const uint32_t hi = ((w[q] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-          // codes 8q .. 8q + 3 and 8q + 4 .. 8q + 7 of the half row: q + 128 - Z in [113, 143],
-          // whose top bit flipped is q - Z as a signed byte
-          o[2 * q] = (__byte_perm(lo, hi, 0x5140) - zc[pp]) ^ 0x80808080u;
-          o[2 * q + 1] = (__byte_perm(lo, hi, 0x7362) - zc[pp]) ^ 0x80808080u;
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t x = w[c], y = w[c] >> 4;
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t sel = static_cast<uint32_t>(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12));
+              o[e] = bf16x2_sub((__byte_perm(x, y, sel) & 0x000F000Fu) | 0x43004300u, zb);
+            }
+            sts128(at + h * kABytes + sw128_off(r, c), make_uint4(o[0], o[1], o[2], o[3]));
+          }
+        } else {
+          uint32_t o[16];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            // codes + 128 in every byte (no byte can borrow from its neighbour below)
+            const uint32_t lo = (w[q] & 0x0F0F0F0Fu) | 0x80808080u;
+            const uint32_t hi = ((w[q] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
+            // codes 8q .. 8q + 3 and 8q + 4 .. 8q + 7 of the half row: q + 128 - Z in
+            // [113, 143], whose top bit flipped is q - Z as a signed byte
+            o[2 * q] = (__byte_perm(lo, hi, 0x5140) - zb) ^ 0x80808080u;
+            o[2 * q + 1] = (__byte_perm(lo, hi, 0x7362) - zb) ^ 0x80808080u;
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            sts128(at + sw128_off(r, 4 * h + c),
+                   make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
         }
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          sts128(at + sw128_off(r, 4 * h + c),
-                 make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
       }
       fence_async_smem();
       __syncwarp();
@@ -312,11 +397,12 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         mbar_arrive(&sb->ld_empty[ls]);
         mbar_arrive(&sb->a_full[os]);
       }
-#pragma unroll
-      for (int pp = 0; pp < kPairs; ++pp) zc[pp] = zn[pp];
+      ld_z(it + kAhead, zq[j]);
+    }
     }
     }
   } else if (warp < 2 + kDecWarps + kPrepWarps) {
+    if constexpr (!kBf) {
     // ------------------------------------------------------------- activation digits
     const int tp = threadIdx.x - 32 * (2 + kDecWarps);  // 0..255
     constexpr int kPrepThreads = 32 * kPrepWarps;
@@ -397,6 +483,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         mbar_arrive(&sb->b_full[os]);
       }
     }
+    }
   } else {
     // ---------------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes 32 quarter .. + 31 (this warp's window)
@@ -405,24 +492,36 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
     const int n = n0 + row;
     const bool live = n < N;
     const int64_t szrow = static_cast<int64_t>(live ? n : 0) * G;
-    // S' of this row two groups ahead (the loads stay in flight across iterations)
-    // (W8A16: the row's scale is applied once, to the finished row)
+    // S' of this row (W8A16: the row's scale is applied once, to the finished row)
     auto ld_s = [&](int it) {
-      if constexpr (kW8) return live ? 1.0f : 0.0f;
+      if constexpr (kW8m) return live ? 1.0f : 0.0f;
       else return it < ng && live ? f16_bits_to_f32(ld_nc_u16(S + szrow + g0 + it)) : 0.0f;
     };
-    float s0 = ld_s(0), s1 = ld_s(1);
-    for (int it = 0; it < ng && !sb->abort; ++it) {
+    float sq[kAhead];
+#pragma unroll
+    for (int j = 0; j < kAhead; ++j) sq[j] = ld_s(j);
+    for (int it0 = 0; it0 < ng && !sb->abort; it0 += kAhead) {
+#pragma unroll
+    for (int j = 0; j < kAhead; ++j) {
+      const int it = it0 + j;
+      if (it >= ng || sb->abort) break;
       const int s = it % kOpStages, b = it % kBufs;
-      const float s2 = ld_s(it + 2);
       if (!sk_wait(&sb->acc_full[b], (it / kBufs) & 1u, sb, status)) break;
       tc_fence_after();
-      const float* meta = reinterpret_cast<const float*>(opst(s) + C::kMetaOff);
-      const float sv = s0;
+      const float* meta = reinterpret_cast<const float*>(opst(s) + C::kMetaOff);  // 2^-s
+      const float sv = sq[j];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * NC;
       constexpr int CH = C::kChunk;
 #pragma unroll
       for (int mc = 0; mc < kEpiTok / CH; ++mc) {
+        if constexpr (kBf) {  // one fp32 column per token: acc += S' D
+          uint32_t d[16];
+          tmem_ld16(taddr + tb + CH * mc, d);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < CH; ++i) acc[CH * mc + i] = fmaf(sv, __uint_as_float(d[i]), acc[CH * mc + i]);
+          continue;
+        }
         uint32_t d0[CH], d1[CH], d2[CH];
         const uint32_t col = tb + CH * mc;
         if constexpr (CH == 16) {
@@ -437,22 +536,22 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
-          const int j = CH * mc + i;
+          const int m = CH * mc + i;
           // |D_i| < 2^21 (2^18 with INT4 codes): digits 0 and 1 combine exactly in 32 bits
           const int d01 = static_cast<int>(d0[i]) + 256 * static_cast<int>(d1[i]);
           const float v = fmaf(65536.0f, static_cast<float>(static_cast<int>(d2[i])),
                                static_cast<float>(d01));
-          acc[j] = fmaf(sv * meta[tb + j], v, acc[j]);
+          acc[m] = fmaf(sv * meta[tb + m], v, acc[m]);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&sb->acc_empty[b]);
-        mbar_arrive(&sb->op_empty[s]);
+        if constexpr (!kBf) mbar_arrive(&sb->op_empty[s]);  // 2^-s read
       }
-      s0 = s1;
-      s1 = s2;
+      sq[j] = ld_s(it + kAhead);
+    }
     }
   }
 
@@ -483,7 +582,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       for (int r = 1; r < 8; ++r)
         if (r < csize) t += v[r];  // rank order
       if (n0 + row < N) {
-        if constexpr (kW8) t *= f16_bits_to_f32(ld_nc_u16(S + n0 + row));
+        if constexpr (kW8m) t *= f16_bits_to_f32(ld_nc_u16(S + n0 + row));
         __nv_bfloat16 hv = __float2bfloat16_rn(t);
         Y[static_cast<int64_t>(m) * ldy + n0 + row] = *reinterpret_cast<uint16_t*>(&hv);
       }
@@ -516,10 +615,12 @@ int pick_split(int tiles, int G, int sms) {
   return best;
 }
 
-template <int MT, bool kW8>
+template <int MT, int kMode>
 cudaError_t launch_mt(const GemvArgs& a, const CUtensorMap& map, int sms, cudaStream_t st) {
-  // activations as [M rows][K] bf16: boxes of 128 k x MT tokens (rows past M read as zero);
-  // kept per thread for the last few activation buffers (decode loops reuse them)
+  // activations as [M rows][K] bf16: boxes of 128 k x MT tokens (rows past M read as zero),
+  // or, as the bf16 MMA operand, 128-byte-swizzled boxes of 64 k x MT tokens; kept per
+  // thread for the last few activation buffers (decode loops reuse them)
+  constexpr bool kBf = kMode == kModeI4Bf;
   struct XEntry {
     const void* p;
     int m, k;
@@ -536,7 +637,7 @@ cudaError_t launch_mt(const GemvArgs& a, const CUtensorMap& map, int sms, cudaSt
     XEntry& e = xcache[xnext];
     e.p = nullptr;
     if (!make_map_2d(&e.map, a.X, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M),
-                     static_cast<uint64_t>(a.ldx) * 2, kGK, MT, false,
+                     static_cast<uint64_t>(a.ldx) * 2, kBf ? 64 : kGK, MT, kBf,
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
       return cudaErrorInvalidValue;
     e.p = a.X;
@@ -546,8 +647,8 @@ cudaError_t launch_mt(const GemvArgs& a, const CUtensorMap& map, int sms, cudaSt
     xnext = (xnext + 1) % kXCache;
     xmap = &e.map;
   }
-  auto kern = tc_skinny_kernel<MT, kW8>;
-  const size_t smem = sk_smem_bytes<MT, kW8>();
+  auto kern = tc_skinny_kernel<MT, kMode>;
+  const size_t smem = sk_smem_bytes<MT, kMode>();
   static std::atomic<bool> attr[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -561,7 +662,7 @@ cudaError_t launch_mt(const GemvArgs& a, const CUtensorMap& map, int sms, cudaSt
   const int cs = pick_split(tiles, G, sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * cs);
-  cfg.blockDim = dim3(SkCfg<MT, kW8>::kThreads);
+  cfg.blockDim = dim3(SkCfg<MT, kMode>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attrs[2];
@@ -610,13 +711,13 @@ const CUtensorMap* weight_map(const void* P, int N, int K, bool w8) {
   return &e.map;
 }
 
-template <bool kW8>
+template <int kMode>
 cudaError_t launch_skinny(const GemvArgs& a, int sms, cudaStream_t st) {
-  const CUtensorMap* map = weight_map(a.P, a.N, a.K, kW8);
+  const CUtensorMap* map = weight_map(a.P, a.N, a.K, kMode == kModeW8);
   if (!map) return cudaErrorInvalidValue;
-  if (a.M <= 16) return launch_mt<16, kW8>(a, *map, sms, st);
-  if (a.M <= 32) return launch_mt<32, kW8>(a, *map, sms, st);
-  return launch_mt<64, kW8>(a, *map, sms, st);
+  if (a.M <= 16) return launch_mt<16, kMode>(a, *map, sms, st);
+  if (a.M <= 32) return launch_mt<32, kMode>(a, *map, sms, st);
+  return launch_mt<64, kMode>(a, *map, sms, st);
 }
 
 bool skinny_common_ok(const GemvArgs& a) {
@@ -633,14 +734,14 @@ bool tc_skinny_ok(const GemvArgs& a) {
 
 cudaError_t launch_tc_skinny(const GemvArgs& a, int sms, cudaStream_t st) {
   if (!tc_skinny_ok(a)) return cudaErrorInvalidValue;
-  return launch_skinny<false>(a, sms, st);
+  return launch_skinny<kModeI4Bf>(a, sms, st);
 }
 
 bool tc_skinny8_ok(const GemvArgs& a) { return skinny_common_ok(a); }
 
 cudaError_t launch_tc_skinny8(const GemvArgs& a, int sms, cudaStream_t st) {
   if (!tc_skinny8_ok(a)) return cudaErrorInvalidValue;
-  return launch_skinny<true>(a, sms, st);
+  return launch_skinny<kModeW8>(a, sms, st);
 }
 
 }  // namespace wq
