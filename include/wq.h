@@ -147,13 +147,11 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
  *   - 9 <= M <= 64 with g = 128 (K % 128 == 0), and 3 <= M <= 8 where the decode kernels
  *     below would pass over the weights more than once (rows too long for blocks of M
  *     tokens): the skinny tensor-core kernel, one pass
- *     over the weights for all tokens. Each token's activations of a group are written as
- *     exact integers x 2^s below 2^22 (s from the group's largest exponent: exact within 2^14
- *     of the group's largest |x|, else off by at most 2^-23 of it) in three signed bytes;
- *     tcgen05 kind::i8 multiplies them with the centred codes q - Z exactly (s32), and
- *     S' 2^-s is applied per group in fp32, so the product is with the exact S'(q - Z). K
- *     is split over a thread-block cluster whose partial rows are summed in a fixed order
- *     (deterministic).
+ *     over the weights for all tokens. tcgen05 kind::f16 multiplies the centred codes
+ *     q - Z (exact in bf16) with the activations as stored, every product exact in fp32 and
+ *     summed in fp32 per group of 128 k, and S' is applied per group in fp32, so the
+ *     product is with the exact S'(q - Z). K is split over a thread-block cluster whose
+ *     partial rows are summed in a fixed order (deterministic).
  *   - otherwise M <= 32: decode kernels, for M > 8 in passes over blocks of at most 8 tokens
  *     (when some block size needs at most 8 passes; else the tensor-core GEMM). The packed rows
  *     stream through shared memory (bulk copies or TMA boxes) or registers, codes are
@@ -179,9 +177,11 @@ wq_status wq_w4a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const uint8_t
 
 /* W8A16 matmul with INT8 symmetric per-channel weights: codes int8 [N, K], S [N]
  * binary16; Y = X (s' q)^T, fp32 accumulation, bf16 out. 3 <= M <= 64 with K % 128 == 0
- * runs on the skinny tensor-core kernel (tcgen05 kind::i8 on the s8 codes as stored and the
- * exact activation digits described for wq_w4a16_gemm; s' applied to the finished row), one
- * pass over the weights; M <= 2 (and other M <= 8) on CUDA cores with the exact s' q; larger
+ * runs on the skinny tensor-core kernel (tcgen05 kind::i8 on the s8 codes as stored and
+ * each token's activations of a group as exact integers x 2^s below 2^22 in three signed
+ * bytes, s from the group's largest exponent: exact within 2^14 of the group's largest |x|,
+ * else off by at most 2^-23 of it; s' applied to the finished row), one pass over the
+ * weights; M <= 2 (and other M <= 8) on CUDA cores with the exact s' q; larger
  * M on the tensor-core GEMM (s' q rounded to bf16). Same requirements as wq_w4a16_gemm. */
 wq_status wq_w8a16_gemm(const uint16_t* X, int64_t M, int64_t ldx, const int8_t* codes,
                         const uint16_t* S, int64_t N, int64_t K, uint16_t* Y, int64_t ldy,

@@ -263,7 +263,8 @@ def test_70b_skinny_sampled(N, K, M):
     """70B-class decode layers at M = 8 and 32 in the benchmark's configuration (the whole W
     quantized and multiplied on the GPU); the oracle quantizes and multiplies 64 sampled rows,
     the first and last among them. Both run on the skinny tensor-core kernel, whose
-    integer products with exact activation digits multiply by the exact S'(q - Z)."""
+    exact bf16 products of the centred codes and the activations, summed in fp32 per group,
+    are scaled by S' per group: the product is with the exact S'(q - Z)."""
     Wb = wq_inputs.weight_bf16(N, K, 0.015)
     Xb = wq_inputs.act_bf16(M, K)
     packed, S, Z = wq.wq_quantize_rtn_g128(gu.bf16_from_bits(Wb))

@@ -1,11 +1,12 @@
-"""Parity of the skinny tensor-core kernel (tcgen05 kind::i8 on exact activation digits,
-split-K over a cluster) with the float64 oracle, through the C ABI: W4A16 (9 to 64 tokens,
-g = 128, centred codes q - Z) on the exact dequantized weights S'(q - Z), and W8A16 (3 to 64
-tokens, the s8 codes copied as they are) on the exact s' q. The W8A16 cases also cover one
+"""Parity of the skinny tensor-core kernel (split-K over a cluster) with the float64 oracle,
+through the C ABI: W4A16 (9 to 64 tokens, g = 128; kind::f16 on the centred codes q - Z as
+bf16 and the activations as stored) on the exact dequantized weights S'(q - Z), and W8A16
+(3 to 64 tokens; kind::i8 on the s8 codes copied as they are and exact activation digits)
+on the exact s' q. The W8A16 cases also cover one
 token, which runs on the row kernel, against the same exact product.
 
 Cases span one group (K = 128, no split), ragged row counts (a partial 128-row tile), every
-token-count class (16, 32, 64 columns per digit plane) with ragged M, long K (70B-class), and
+token-count class (16, 32, 64 token columns) with ragged M, long K (70B-class), and
 outlier activations (a token's group scale set by one large channel)."""
 import numpy as np
 import pytest

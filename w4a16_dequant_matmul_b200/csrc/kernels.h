@@ -60,8 +60,9 @@ int gemv_fast_block(const GemvArgs& a);
 cudaError_t launch_gemv_stream(const GemvArgs& a, int sms, cudaStream_t st);
 cudaError_t launch_gemv_w4a16(const GemvArgs& a, int sms, cudaStream_t st);
 
-// Skinny M (up to kSkinnyMaxTokens tokens), g = 128: tcgen05 kind::i8 on the codes and exact
-// activation digits, split-K over a thread-block cluster (tc_skinny.cu). a.M is the full M.
+// Skinny M (up to kSkinnyMaxTokens tokens), g = 128: tcgen05 kind::f16 on the centred codes
+// as bf16 and the activations, split-K over a thread-block cluster (tc_skinny.cu). a.M is the
+// full M.
 constexpr int kSkinnyMaxTokens = 64;
 bool tc_skinny_ok(const GemvArgs& a);
 cudaError_t launch_tc_skinny(const GemvArgs& a, int sms, cudaStream_t st);

@@ -1,35 +1,42 @@
-// Skinny W4A16 matmul (a handful to 64 tokens) on the 5th-generation tensor core with exact
-// integer arithmetic: Y = X W_hat^T, g = 128.
+// Skinny W4A16 / W8A16 matmul (a handful to 64 tokens) on the 5th-generation tensor core:
+// Y = X W_hat^T, the weights read once for every token count.
 // ("LLM Weight Quantization - GPTQ, AWQ, SmoothQuant, FP8 & INT4/INT8 Trade-offs",
 // "The vocabulary": 4-bit weights, 16-bit activations, fp32 accumulation; "Overview": decode
 // reads every weight once.)
 //
-// Per group of 128 k and weight row n,
-//     sum_k x_k S'(q_k - Z) = S' 2^-s sum_i 2^(8i) D_i,
-// where, per token, x_k 2^s is rounded to an integer below 2^22 in magnitude (s from the
-// token's largest exponent in the group: exact within 2^14 of the group's largest |x|, else
-// off by at most 2^-23 of it) and split into three signed bytes d_i (balanced digits), and
-// D_i = sum_k (q_k - Z) d_i,k are exact s32 dot products. The centred codes q - Z (in
-// [-15, 15]) are the MMA's A operand (M = 128 weight rows, s8), the digits its B operand
-// (N = 3 MT columns: digit plane i of token m is column i MT + m, s8), one tcgen05.mma
-// kind::i8 per 32 k, four per group, into a fresh TMEM accumulator. A tcgen05.mma costs the same issue time for any
-// N up to 256, so all tokens share each instruction: the weights are read once for every M.
+// INT4, g = 128. Per group of 128 k and weight row n,
+//     sum_k x_k S'(q_k - Z) = S' D,   D = sum_k (q_k - Z) x_k,
+// where the centred codes q - Z (integers in [-15, 15], exact in bf16) are the MMA's A
+// operand (M = 128 weight rows) and the activations, bf16 as stored, its B operand
+// (N = MT token columns): eight tcgen05.mma kind::f16 (K = 16) per group into a fresh fp32
+// TMEM accumulator. Every product is exact in fp32; D is their fp32 sum, and the epilogue
+// adds S' D into the row's fp32 accumulators.
+//
+// W8A16 (s' per row): per group, sum_k x_k q_k = 2^-s sum_i 2^(8i) D_i, where per token x_k 2^s
+// is rounded to an integer below 2^22 in magnitude (s from the token's largest exponent in the
+// group: exact within 2^14 of the group's largest |x|, else off by at most 2^-23 of it) and
+// split into three signed bytes d_i (balanced digits), and D_i = sum_k q_k d_i,k are exact
+// s32 dot products: the s8 codes are A (copied by TMA as stored), the digit planes B
+// (N = 3 MT columns), one tcgen05.mma kind::i8 per 32 k; s' multiplies the finished row.
 //
 // A CTA owns a 128-row tile and a contiguous range of its groups; the CTAs of a cluster
 // split K and sum their partial rows through distributed shared memory in rank order
 // (deterministic). Warp roles per CTA:
-//   warp 0       TMA producer: per group, the tile's packed codes ([128 rows x 64 B] box)
-//                and the activations ([MT tokens x 128 k] bf16 box) into a ring of stages;
+//   warp 0       TMA producer. INT4: per group, the tile's packed codes ([128 rows x 64 B]
+//                box) into the load ring, and the activations (two 128-byte-swizzled
+//                [MT tokens x 64 k] bf16 boxes) into the operand stage. W8A16: the s8 code
+//                box (128-byte swizzled) into the operand stage, the activations
+//                ([MT tokens x 128 k]) into the load ring;
 //   warp 1       TMEM allocation; lane 0 issues the MMAs of a group once its A and B tiles
-//                are written and a TMEM buffer is free, commits the stage and the buffer;
-//   next 8 (4 at MT = 64) warps: code expansion: each thread turns half rows (32 packed
-//                bytes each) into centred s8 codes q - Z in the 128-byte-swizzled K-major A
-//                tile;
-//   next 8 warps activation digits: 8 threads per token, 16 k each: the group's exponent,
-//                the digit planes into the swizzled B tile, and 2^-s;
+//                are in place and a TMEM accumulator is free, commits the stage and the
+//                accumulator;
+//   INT4: 8 warps of code expansion: each thread turns a half row (32 packed bytes) into
+//                bf16 pairs q - Z in the 128-byte-swizzled K-major A tile (two atoms);
+//   W8A16: 8 warps of activation digits: 8 threads per token, 16 k each: the group's
+//                exponent, the digit planes into the swizzled B tile, and 2^-s;
 //   last 4 (8 at MT = 64) warps  epilogue: thread = TMEM lane = weight row (at MT = 64 two
-//                warps per lane quarter, each for half the tokens); reads the three digit planes of
-//                the group's accumulator, combines them, applies S' 2^-s, accumulates fp32.
+//                warps per lane quarter, each for half the tokens); reads the group's
+//                accumulator columns, scales them, accumulates fp32.
 // Every mbarrier wait is bounded (2 s): on a timeout the kernel records kStTimeout, every role
 // leaves its loop, the producer waits (bounded) for its copies, the MMA lane for its last
 // commit, and the CTA frees TMEM and returns.
@@ -59,7 +66,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kAhead = 8;
 
 // Operand modes:
-//   kModeI4Dig  INT4 codes: centred codes q - Z as s8 x activation digit planes (kind::i8).
 //   kModeW8     INT8 symmetric per-channel weights (W8A16): the s8 codes are the A operand
 //               as they are. The producer copies each [128 rows x 128 k] box with TMA
 //               straight into the operand stage in the 128-byte-swizzled layout, so there is
@@ -69,7 +75,7 @@ constexpr int kAhead = 8;
 //               product is exact in fp32). The producer copies X with TMA straight into the
 //               operand stage (two 128-byte-swizzled boxes of 64 k per group), so there is no
 //               digit role, and the epilogue applies S' to one accumulator column per token.
-enum SkMode { kModeI4Dig = 0, kModeW8 = 1, kModeI4Bf = 2 };
+enum SkMode { kModeW8 = 1, kModeI4Bf = 2 };
 
 template <int MT, int kMode>
 struct SkCfg {
@@ -90,9 +96,8 @@ struct SkCfg {
   static constexpr int kLdStages = MT <= 16 ? 6 : (MT <= 32 ? (kBf ? 6 : 5) : 3);
   static constexpr int kBufs = (kBf || MT <= 32) ? 4 : 2;  // TMEM accumulators in flight
   static constexpr int kChunk = (kBf || MT <= 16) ? 16 : 8;  // tokens per epilogue TMEM load
-  // code-expansion warps: 8 (one half row per thread), or 4 (two) where the epilogue's MT
-  // accumulators need the registers of a smaller block
-  static constexpr int kDecWarps = kW8m ? 0 : ((kBf || MT <= 32) ? 8 : 4);
+  // code-expansion warps (INT4): 8, one half row per thread
+  static constexpr int kDecWarps = kW8m ? 0 : 8;
   static constexpr int kPrepWarps = kBf ? 0 : 8;  // activation digits
   // epilogue warps: one per TMEM lane quarter, or two at MT = 64, each then keeping the
   // accumulators of half the tokens (32 registers instead of 64)
@@ -296,26 +301,18 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       if (!mbar_wait_bounded(&sb->done, 0, kLimitNs)) set_status(status, kStTimeout);
     }
   } else if (warp < 2 + kDecWarps) {
-    if constexpr (!kW8m) {
+    if constexpr (kBf) {
     // --------------------------------------------------------------- code expansion
-    // s8 codes: thread t takes the half rows (row, half) = pair >> 1, pair & 1 for pairs
-    // t, t + 32 kDecWarps, ...: a quarter-warp reads 256 contiguous bytes of the raw tile,
-    // and each 16-byte store of the eight lands in a distinct slot. bf16 codes (half h of a
-    // row is the row of atom h): the 8 threads of a quarter-warp take 8 consecutive rows
-    // (distinct store slots) and both halves (reads spread over 4 slots); the quarter-warp
-    // after it takes the same rows' other halves.
+    // Half h of a row (64 k) is that row of A's atom h. The 8 threads of a quarter-warp take
+    // 8 consecutive rows (distinct store slots) and both halves (reads spread over 4 slots);
+    // the quarter-warp after it takes the same rows' other halves.
     constexpr int kPairs = 256 / (32 * kDecWarps);
     const int t = threadIdx.x - 64;
     const int G = K / kGK;
     auto pair_rh = [&](int pp, int& r, int& h) {
       const int pr = t + 32 * kDecWarps * pp;
-      if constexpr (kBf) {
-        r = 8 * (pr >> 4) + (pr & 7);
-        h = ((pr >> 3) & 1) ^ ((pr >> 1) & 1);
-      } else {
-        r = pr >> 1;
-        h = pr & 1;
-      }
+      r = 8 * (pr >> 4) + (pr & 7);
+      h = ((pr >> 3) & 1) ^ ((pr >> 1) & 1);
     };
     int64_t zrow[kPairs];
 #pragma unroll
@@ -325,7 +322,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
       const int n = n0 + r;
       zrow[pp] = n < N ? static_cast<int64_t>(n) * G : -1;  // rows past N: codes and Z are 0
     }
-    // Z of the rows, in every byte (s8) or as 128 + Z in both bf16 halves
+    // Z of the rows, as 128 + Z in both bf16 halves
     auto ld_z = [&](int it, uint32_t (&z4)[kPairs]) {
 #pragma unroll
       for (int pp = 0; pp < kPairs; ++pp) {
@@ -333,7 +330,7 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
             it < ng && zrow[pp] >= 0
                 ? static_cast<uint32_t>(f16_bits_to_f32(ld_nc_u16(Zp + zrow[pp] + g0 + it)))
                 : 0u;
-        z4[pp] = kBf ? z * 0x00010001u + 0x43004300u : z * 0x01010101u;
+        z4[pp] = z * 0x00010001u + 0x43004300u;
       }
     };
     uint32_t zq[kAhead][kPairs];
@@ -358,37 +355,19 @@ tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
         const uint4 p0 = lds128(raw + r * 64 + 32 * h), p1 = lds128(raw + r * 64 + 32 * h + 16);
         const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
         const uint32_t zb = zq[j][pp];  // Z of this group (ring slot j)
-        if constexpr (kBf) {
-          // word c = codes 8c .. 8c + 7 of the half row = 16-byte chunk c of its atom row.
-          // bf16 pair e: byte e of the word (low half) and of the word >> 4 (high half), low
-          // nibbles kept and 0x4300 set: 128 + code exactly; minus 128 + Z: q - Z exactly.
+        // word c = codes 8c .. 8c + 7 of the half row = 16-byte chunk c of its atom row.
+        // bf16 pair e: byte e of the word (low half) and of the word >> 4 (high half), low
+        // nibbles kept and 0x4300 set: 128 + code exactly; minus 128 + Z: q - Z exactly.
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t x = w[c], y = w[c] >> 4;
-            uint32_t o[4];
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t x = w[c], y = w[c] >> 4;
+          uint32_t o[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t sel = static_cast<uint32_t>(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12));
-              o[e] = bf16x2_sub((__byte_perm(x, y, sel) & 0x000F000Fu) | 0x43004300u, zb);
-            }
-            sts128(at + h * kABytes + sw128_off(r, c), make_uint4(o[0], o[1], o[2], o[3]));
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t sel = static_cast<uint32_t>(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12));
+            o[e] = bf16x2_sub((__byte_perm(x, y, sel) & 0x000F000Fu) | 0x43004300u, zb);
           }
-        } else {
-          uint32_t o[16];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            // codes + 128 in every byte (no byte can borrow from its neighbour below)
-            const uint32_t lo = (w[q] & 0x0F0F0F0Fu) | 0x80808080u;
-            const uint32_t hi = ((w[q] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-            // codes 8q .. 8q + 3 and 8q + 4 .. 8q + 7 of the half row: q + 128 - Z in
-            // [113, 143], whose top bit flipped is q - Z as a signed byte
-            o[2 * q] = (__byte_perm(lo, hi, 0x5140) - zb) ^ 0x80808080u;
-            o[2 * q + 1] = (__byte_perm(lo, hi, 0x7362) - zb) ^ 0x80808080u;
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            sts128(at + sw128_off(r, 4 * h + c),
-                   make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
+          sts128(at + h * kABytes + sw128_off(r, c), make_uint4(o[0], o[1], o[2], o[3]));
         }
       }
       fence_async_smem();
