@@ -8,17 +8,21 @@
 // (persistent, one per SM), warp roles:
 //   warp 0      TMA producer: X tiles [256 tokens x 64 k] bf16, 128-byte swizzle, into the
 //               stage ring (completes on the stage's "full" mbarrier).
-//   warp 1      allocates TMEM (512 columns = two 128 x 256 fp32 accumulators); lane 0
-//               issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32), 4 per stage, and
-//               commits each stage to its "empty" barrier and each tile to "acc_full".
-//   warps 2-9   dequantizers: thread (h, r) owns half h of weight row r of the stage; it
-//               keeps the packed bytes and S', Z of the next two stages in flight, forms
+//   warp 1      allocates TMEM (512 columns: one 128 x 256 fp32 accumulator, then the A
+//               tile of every stage, 32 columns each); lane 0 issues tcgen05.mma
+//               (kind::f16, A from tensor memory, B from shared memory, fp32 accumulation),
+//               4 per stage, and commits each stage to its "empty" barrier and each tile to
+//               "acc_full".
+//   warps 2-9   dequantizers: thread (h, r) owns half h of weight row r of the stage (r is
+//               its TMEM lane); it keeps S', Z of the next two stages in flight, forms
 //               W_hat = S'(q - Z) exactly in fp32 (one byte-permute per weight, packed
-//               fp32x2 FMAs), rounds to bf16 and writes its 32 values into the A tile in
-//               the canonical K-major 128-byte-swizzled layout.
+//               fp32x2 FMAs), rounds to bf16 and writes its 32 values as 16 bf16 pairs into
+//               its TMEM lane of the stage's A columns (tcgen05.st), so the dequantized
+//               tile never passes through shared memory.
 //   warps 10-13 epilogue: tcgen05.ld the accumulator (32 rows per warp, its TMEM lane
-//               quarter), round to bf16, stage [256 tokens x 128 rows] in shared memory
-//               and write it to Y with one TMA store per tile.
+//               quarter), round to bf16, stage [32 tokens x 128 rows] in shared memory and
+//               write it to Y with one TMA store per 32 tokens; the next tile's MMAs start
+//               once the accumulator has been read.
 // Every mbarrier wait is bounded (2 s): on a timeout the kernel records kStTimeout and all
 // roles leave their loops; the TMA lane waits (bounded) for the copies it issued, the MMA
 // lane for its last commit, and the CTA frees TMEM and exits.
@@ -36,34 +40,40 @@ namespace {
 constexpr int kRows = 128;     // weight rows per tile (MMA M)
 constexpr int kToks = 256;     // tokens per tile (MMA N)
 constexpr int kBK = 64;        // k per stage (one 128-byte swizzle atom of bf16)
-constexpr int kABytes = kRows * kBK * 2;    // 16 KB: dequantized bf16 weight tile
 constexpr int kBBytes = kToks * kBK * 2;    // 32 KB: X tile
-constexpr int kEpiToks = 64;                // tokens per epilogue store
-constexpr int kEpiBytes = kEpiToks * kRows * 2;  // 16 KB
-// Stage ring depth and raw-code bytes per stage: INT4 keeps 32 B/row, INT8 64 B/row.
+constexpr int kEpiToks = 32;                // tokens per epilogue store
+constexpr int kEpiBytes = kEpiToks * kRows * 2;  // 8 KB
+// Stage ring depth and raw-code bytes per stage: INT4 keeps 32 B/row, INT8 64 B/row. The
+// dequantized weight tile of a stage lives in tensor memory, so shared memory holds only
+// the X tile and the raw codes per stage: six stages (five for INT8) cover the copies'
+// latency.
 template <bool kInt8> struct Cfg {
   static constexpr int kRBytes = kRows * (kInt8 ? kBK : kBK / 2);
-  static constexpr int kStages = kInt8 ? 3 : 4;
+  static constexpr int kStages = kInt8 ? 5 : 6;
 };
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kThreads = 448;  // 14 warps: TMA, MMA, 8 dequant, 4 epilogue
 constexpr int kDqWarps = 8;
+// TMEM: the 128 x 256 fp32 accumulator in columns 0..255, then per stage the A tile
+// (128 lanes x 64 k as bf16 pairs = 32 columns).
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kACol0 = kToks;
+static_assert(kACol0 + 32 * kMaxStages <= kTmemCols, "TMEM");
 constexpr uint64_t kLimitNs = 2000000000ull;
 
 struct Smem {
   uint64_t raw_full[kMaxStages];  // TMA: X tile + raw weight codes landed (tx bytes)
   uint64_t full[kMaxStages];      // dequant warps: bf16 weight tile written
   uint64_t empty[kMaxStages];     // tcgen05.commit: the stage's MMAs are done
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t acc_full;   // the tile's accumulator is complete
+  uint64_t acc_empty;  // the epilogue has read it
   uint64_t done;
   uint32_t tmem_base;
   volatile int abort;
 };
 template <bool kInt8>
 constexpr size_t smem_bytes() {
-  return 1024 + Cfg<kInt8>::kStages * (kABytes + kBBytes + Cfg<kInt8>::kRBytes) + kEpiBytes +
+  return 1024 + Cfg<kInt8>::kStages * (kBBytes + Cfg<kInt8>::kRBytes) + kEpiBytes +
          sizeof(Smem);
 }
 
@@ -77,17 +87,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm
   set_status(status, kStTimeout);
   atomicExch(const_cast<int*>(&sm->abort), 1);
   return false;
-}
-
-// Dequantize 64 codes of one row (32 packed bytes, or 64 int8 bytes) into 8 chunks of 8
-// bf16 values and store them into the swizzled A tile row.
-__device__ __forceinline__ void store_row_chunk(uint32_t tile, int r, int c, const float* w) {
-  uint4 v;
-  v.x = pack_bf16x2(w[0], w[1]);
-  v.y = pack_bf16x2(w[2], w[3]);
-  v.z = pack_bf16x2(w[4], w[5]);
-  v.w = pack_bf16x2(w[6], w[7]);
-  sts128(tile + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4), v);
 }
 
 // Eight codes of a 32-bit word (nibble i = code of k = i) -> S'(q - Z), exact in fp32:
@@ -129,8 +128,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* tileA = base;                              // [kStages][kABytes]
-  uint8_t* tileB = base + kStages * kABytes;          // [kStages][kBBytes]
+  uint8_t* tileB = base;                              // [kStages][kBBytes]
   uint8_t* tileR = tileB + kStages * kBBytes;         // [kStages][kRBytes]
   uint8_t* epi = tileR + kStages * kRBytes;           // [kEpiToks][kRows] bf16
   Smem* sm = reinterpret_cast<Smem*>(epi + kEpiBytes);
@@ -148,10 +146,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
       mbar_init(&sm->full[s], kDqWarps);    // dequant warps
       mbar_init(&sm->empty[s], 1);     // tcgen05.commit
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm->acc_full[b], 1);
-      mbar_init(&sm->acc_empty[b], 4);
-    }
+    mbar_init(&sm->acc_full, 1);
+    mbar_init(&sm->acc_empty, 4);
     mbar_init(&sm->done, 1);
     sm->abort = 0;
     fence_barrier_init();
@@ -199,10 +195,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     if (lane == 0) {
       uint32_t it = 0, j = 0;
       for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x, ++j) {
-        const int b = j & 1;
-        if (j >= 2 && !wait_or_abort(&sm->acc_empty[b], ((j >> 1) - 1) & 1u, sm, status)) break;
+        if (j >= 1 && !wait_or_abort(&sm->acc_empty, (j - 1) & 1u, sm, status)) break;
         tc_fence_after();
-        const uint32_t d = tmem + b * kToks;
+        const uint32_t d = tmem;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kStages;
@@ -212,16 +207,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             break;
           }
           tc_fence_after();
-          const uint8_t* a = tileA + s * kABytes;
+          const uint32_t a = tmem + kACol0 + 32 * s;  // A: 8 TMEM columns per K = 16
           const uint8_t* bt = tileB + s * kBBytes;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
-            tc_mma(d, sw128_desc(a + 32 * k), sw128_desc(bt + 32 * k), kIdesc,
-                   (kb | k) != 0 ? 1u : 0u);
+            tc_mma_tmem_a(d, a + 8 * k, sw128_desc(bt + 32 * k), kIdesc, (kb | k) != 0 ? 1u : 0u);
           tc_commit(&sm->empty[s]);
         }
         if (!ok) break;
-        tc_commit(&sm->acc_full[b]);
+        tc_commit(&sm->acc_full);
       }
       // all issued MMAs have completed once this commit arrives
       tc_commit(&sm->done);
@@ -229,12 +223,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     }
   } else if (warp < 2 + kDqWarps) {
     // ------------------------------------------------------------------ dequantizers
-    // Lane pairs share a weight row: thread (r, h) handles half h (32 k) of row r, so a
-    // quarter-warp reads 128 contiguous bytes of the raw tile and writes 8 distinct
-    // 16-byte slots of the swizzled A tile (both bank-conflict free).
-    const int td = threadIdx.x - 64;                  // 0..255
-    const int r = (td >> 5) * 16 + ((td & 31) >> 1);  // weight row within the tile
-    const int h = td & 1;                             // which 32-k half of the stage
+    // Thread = weight row r of the tile (its warp's TMEM lane quarter, its lane) and half h
+    // (32 k) of the stage: it writes its 16 bf16 pairs into TMEM lane r, columns 16 h ..
+    // 16 h + 15 of the stage's A tile.
+    const int quarter = warp & 3;
+    const int h = (warp - 2) >> 2;                    // which 32-k half of the stage
+    const int r = quarter * 32 + lane;                // weight row within the tile
+    const uint32_t a_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kACol0 + 16 * h;
     // (tile, kb) of the iteration whose scales are fetched next, advanced incrementally
     int f_t = blockIdx.x, f_kb = 0;
     auto fetch = [&](float& fa, float& fc) {
@@ -261,7 +256,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     float a0, c0, a1, c1;
     fetch(a0, c0);
     fetch(a1, c1);
-    const uint32_t tileA_s = smem_u32(tileA), tileR_s = smem_u32(tileR);
+    const uint32_t tileR_s = smem_u32(tileR);
     uint32_t it = 0;
     for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x) {
       bool ok = true;
@@ -273,11 +268,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         const int s = it % kStages;
         const uint32_t u = it / kStages;
         // the raw codes of this stage have landed (which also means the stage's previous
-        // MMAs are done, since the TMA for it was issued only after "empty")
+        // MMAs, which read its A columns, are done: the TMA for it was issued only after
+        // "empty")
         if (!wait_or_abort(&sm->raw_full[s], u & 1u, sm, status)) {
           ok = false;
           break;
         }
+        tc_fence_after();
         const uint32_t raw = tileR_s + s * kRBytes;
         float w[32];
         if (!kInt8) {
@@ -292,10 +289,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
 #pragma unroll
           for (int q = 0; q < 8; ++q) dq4_int8(words[q], ca, w + 4 * q);
         }
-        const uint32_t tile = tileA_s + s * kABytes;
+        uint32_t v[16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) store_row_chunk(tile, r, 4 * h + c, w + 8 * c);
-        fence_async_smem();
+        for (int i = 0; i < 16; ++i) v[i] = pack_bf16x2(w[2 * i], w[2 * i + 1]);
+        tmem_st16(a_lane + 32 * s, v);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->full[s]);
       }
@@ -309,8 +308,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     uint32_t j = 0;
     for (int t = blockIdx.x; t < tiles && !sm->abort; t += gridDim.x, ++j) {
       const int nt = t / m_tiles, mt = t % m_tiles;
-      const int b = j & 1;
-      if (!wait_or_abort(&sm->acc_full[b], (j >> 1) & 1u, sm, status)) break;
+      if (!wait_or_abort(&sm->acc_full, j & 1u, sm, status)) break;
       tc_fence_after();
       const uint32_t st = smem_u32(epi);
       for (int hf = 0; hf < kToks / kEpiToks; ++hf) {
@@ -318,9 +316,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         named_barrier(2, 128);
         for (int c = 0; c < kEpiToks / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + b * kToks +
-                        hf * kEpiToks + c * 32,
-                    v);
+          tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + hf * kEpiToks + c * 32, v);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -331,7 +327,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         if (hf == kToks / kEpiToks - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
+          if (lane == 0) mbar_arrive(&sm->acc_empty);
         }
         fence_async_smem();
         named_barrier(2, 128);
