@@ -162,7 +162,7 @@ wq_status wq_dequant(const uint8_t* packed, const uint16_t* S, const uint16_t* Z
  *     K % 128 == 0, N % 32 == 0 or N % 16 == 0, 16-byte aligned X, S, Z, and X plus one
  *     tile's S' and Z within shared memory); otherwise it runs on the tensor-core GEMM.
  *   - larger M: the tcgen05/TMEM tensor-core GEMM, which dequantizes each weight tile to
- *     bf16 in shared memory (so W_hat is rounded to bfloat16 there, then multiplied
+ *     bf16 in tensor memory (so W_hat is rounded to bfloat16 there, then multiplied
  *     exactly with fp32 accumulation).
  * Requirements: K % 32 == 0; g a multiple of 32 dividing K, or 0; X 16-byte aligned and
  * ldx % 8 == 0; packed 16-byte aligned; S, Z, Y 2-byte aligned. On the tensor-core path
