@@ -6,8 +6,9 @@
 // Tile: 128 weight rows (MMA M) x 256 tokens (MMA N), K in stages of 64. The weight tile is
 // the MMA's A operand so that a dequantized tile feeds 256 tokens at once. Per CTA
 // (persistent, one per SM), warp roles:
-//   warp 0      TMA producer: X tiles [256 tokens x 64 k] bf16, 128-byte swizzle, into the
-//               stage ring (completes on the stage's "full" mbarrier).
+//   warp 0      TMA producer: X tiles [256 tokens x 64 k] bf16, 128-byte swizzle, and the
+//               tile's raw codes of the same 64 k into the stage ring (both complete on the
+//               stage's "raw_full" mbarrier); a stage is refilled once its MMAs are done.
 //   warp 1      allocates TMEM (512 columns: one 128 x 256 fp32 accumulator, then the A
 //               tile of every stage, 32 columns each); lane 0 issues tcgen05.mma
 //               (kind::f16, A from tensor memory, B from shared memory, fp32 accumulation),
