@@ -1,4 +1,5 @@
-"""Model check of the barrier protocol of the tensor-core prefill GEMM (tc_gemm.cu).
+"""Model checks of the barrier protocols of the tensor-core kernels: the prefill GEMM
+(tc_gemm.cu) and, at the end, the skinny kernel's INT4 form (tc_skinny.cu).
 
 The dequantized weight tile of each stage lives in tensor memory, in columns tied to the
 stage of the shared-memory ring, and one accumulator serves every tile. The kernel's roles
@@ -201,6 +202,142 @@ def test_gemm_model_catches_missing_empty_wait():
     for seed in range(30):
         try:
             run_gemm_protocol(3, 4, 2, NW=2, NE=1, seed=seed, producer_waits_empty=False)
+        except (AssertionError, IndexError, RuntimeError):
+            caught += 1
+    assert caught > 0
+
+
+def run_skinny_protocol(groups, LS, OS, NB, NW, NE, seed, expansion_waits_op_empty=True):
+    """The skinny tensor-core kernel's INT4 form (tc_skinny.cu), one CTA:
+
+    producer   per group i: wait ld_empty[i % LS], copy the packed codes -> ld_full; wait
+               op_empty[i % OS], copy the activations into the operand stage -> b_full
+    expansion  NW warps; per group: wait ld_full and op_empty, write A into the operand
+               stage, arrive ld_empty and a_full
+    MMA lane   per group: wait a_full, b_full and acc_empty[i % NB], issue, commit op_empty
+               and acc_full[i % NB]
+    epilogue   NE warps; per group: wait acc_full, read the accumulator, arrive acc_empty
+    """
+    rnd = random.Random(seed)
+    ld_full = [Bar(1) for _ in range(LS)]
+    ld_empty = [Bar(NW) for _ in range(LS)]
+    a_full = [Bar(NW) for _ in range(OS)]
+    b_full = [Bar(1) for _ in range(OS)]
+    op_empty = [Bar(1) for _ in range(OS)]
+    acc_full = [Bar(1) for _ in range(NB)]
+    acc_empty = [Bar(NE) for _ in range(NB)]
+    inflight, mma_fifo = [], []
+    reading = [0] * OS
+    a_of = [None] * OS
+    a_writes = [0] * OS
+    acc_of = [None] * NB
+    epi_reads = [0] * groups
+
+    def producer():
+        for i in range(groups):
+            s, u = i % LS, i // LS
+            if u > 0:
+                while not ld_empty[s].ready((u - 1) & 1):
+                    yield
+            ld_full[s].expect(("codes", i), 1)
+            inflight.append((ld_full[s], 1))
+            yield
+            o, ou = i % OS, i // OS
+            if ou > 0:
+                while not op_empty[o].ready((ou - 1) & 1):
+                    yield
+            b_full[o].expect(("x", i), 1)
+            inflight.append((b_full[o], 1))
+            yield
+
+    def expansion():
+        for i in range(groups):
+            s, u, o, ou = i % LS, i // LS, i % OS, i // OS
+            while not ld_full[s].ready(u & 1):
+                yield
+            if ou > 0 and expansion_waits_op_empty:
+                while not op_empty[o].ready((ou - 1) & 1):
+                    yield
+            assert len(ld_full[s].fills) - 1 == u and ld_full[s].fills[u] == ("codes", i)
+            assert reading[o] == 0, ("A rewritten under a queued MMA", i)
+            if a_of[o] != i:
+                a_of[o], a_writes[o] = i, 0
+            a_writes[o] += 1
+            yield
+            ld_empty[s].arrive()
+            a_full[o].arrive()
+
+    def mma():
+        for i in range(groups):
+            o, ou, b, v = i % OS, i // OS, i % NB, i // NB
+            while not (a_full[o].ready(ou & 1) and b_full[o].ready(ou & 1)):
+                yield
+            if v > 0:
+                while not acc_empty[b].ready((v - 1) & 1):
+                    yield
+            assert a_of[o] == i and a_writes[o] == NW, ("MMA on an unfinished A", i)
+            assert len(b_full[o].fills) - 1 == ou and b_full[o].fills[ou] == ("x", i)
+            assert v == 0 or epi_reads[i - NB] == NE, ("accumulator overwritten", i)
+            acc_of[b] = i
+            reading[o] += 1
+            mma_fifo.append((o, i, b))
+            yield
+
+    def epilogue():
+        for i in range(groups):
+            b, v = i % NB, i // NB
+            while not acc_full[b].ready(v & 1):
+                yield
+            assert acc_full[b].fills[v] == ("acc", i) and acc_of[b] == i
+            yield
+            epi_reads[i] += 1
+            acc_empty[b].arrive()
+
+    def complete_mma():
+        o, i, b = mma_fifo.pop(0)
+        reading[o] -= 1
+        op_empty[o].arrive()
+        acc_full[b].arrive(("acc", i))
+
+    alive = ([producer(), mma()] + [expansion() for _ in range(NW)] +
+             [epilogue() for _ in range(NE)])
+    steps = 0
+    while alive or inflight or mma_fifo:
+        steps += 1
+        if steps > 500000:
+            raise RuntimeError("deadlock")
+        r = rnd.random()
+        if inflight and (not alive or r < 0.25):
+            bar, tx = inflight.pop(rnd.randrange(len(inflight)))
+            bar.land(tx)
+            continue
+        if mma_fifo and (not alive or r < 0.45):
+            complete_mma()
+            continue
+        if not alive:
+            continue
+        g = rnd.choice(alive)
+        try:
+            next(g)
+        except StopIteration:
+            alive.remove(g)
+    assert epi_reads == [NE] * groups
+
+
+@pytest.mark.parametrize("groups", [1, 3, 8, 17])
+@pytest.mark.parametrize("LS,OS,NB", [(6, 4, 4), (2, 2, 1), (3, 5, 2)])
+def test_skinny_protocol_random_schedules(groups, LS, OS, NB):
+    for seed in range(4):
+        run_skinny_protocol(groups, LS, OS, NB, NW=3, NE=2, seed=seed * 6007 + groups)
+
+
+def test_skinny_model_catches_missing_op_empty_wait():
+    """Planted mistake: the expansion warps write a stage's A without waiting for the MMAs
+    that read its previous contents; the model must see A rewritten under a queued MMA."""
+    caught = 0
+    for seed in range(30):
+        try:
+            run_skinny_protocol(9, 4, 2, 2, NW=2, NE=1, seed=seed, expansion_waits_op_empty=False)
         except (AssertionError, IndexError, RuntimeError):
             caught += 1
     assert caught > 0
